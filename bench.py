@@ -1,0 +1,401 @@
+"""Benchmark of route-layer chunk-routing sparse attention on B200.
+
+One step = one route layer over one synthetic sequence: rdl_summary_pool +
+rdl_route_score_topk + rdl_route_attn on the 16K Dream-7B-shaped prefill (28 query heads,
+4 KV heads, head dim 128, K = 32 chunks, window radius 256, rank-64 residual), inputs
+resident in HBM.  The metric is route-layer query tokens per second (content rows; the
+mask-slot rows are produced by the summary pool inside the same step).  The JSON line
+also carries the 128K decode block (score + attention with cached summaries, ms per step).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun every rank processes its own sequence (no exchange between ranks), the
+timed region is bracketed by barriers and the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "route-layer sparse-attn query-tokens/s at 16K-128K; decode-step ms at 128K"
+UNIT = "query-tokens/s"
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def attn_flops(dims, q_pos, idx) -> float:
+    """2 (QK) + 2 (PV) flops x d per attended key per (row, head): window keys |W(p)| and
+    the 63 content keys of each selected chunk, content rows only."""
+    L, w, d, Hq, Hkv = dims.L, dims.w, dims.d, dims.Hq, dims.Hkv
+    G = Hq // Hkv
+    pos = np.arange(L) if q_pos is None else np.asarray(q_pos[0], dtype=np.int64)
+    content = (pos % 64) != 63
+    win = np.minimum(L, pos + w + 1) - np.maximum(0, pos - w) if w >= 0 else np.zeros_like(pos)
+    nsel = (idx[0] >= 0).sum(axis=-1)                       # [Hkv, Lq]
+    keys = (win[None, :] + 63 * nsel) * content[None, :]    # per (group, row)
+    return float(4 * d * G * keys.sum())
+
+
+def score_flops(dims) -> float:
+    Lq, C = dims.Lq, dims.L // 64
+    return float(2 * Lq * dims.D * dims.r + 2 * Lq * dims.r * dims.Hq * dims.d
+                 + 2 * Lq * dims.Hq * C * dims.d)
+
+
+def decode_bytes(dims, idx) -> dict:
+    """Bytes a decode step must move: summaries + entropies, every distinct selected
+    (group, chunk) K/V slab, the window K/V, the queries, residual inputs and outputs."""
+    C = dims.L // 64
+    s_bytes = 4 * dims.B * dims.Hq * C * (dims.d + 1)
+    uniq = sum(len(set(idx[b, g][idx[b, g] >= 0].tolist())) for b in range(idx.shape[0])
+               for g in range(idx.shape[1]))
+    chunk_bytes = uniq * 2 * 64 * dims.d * 2
+    win_keys = min(dims.L, 64 + 2 * dims.w)                 # union of the block's windows
+    win_bytes = dims.B * dims.Hkv * win_keys * 2 * dims.d * 2
+    io = 2 * dims.B * dims.Lq * (2 * dims.Hq * dims.d + dims.D) + 2 * (dims.D * dims.r
+                                                                       + dims.r * dims.Hq * dims.d)
+    return {"total": s_bytes + chunk_bytes + win_bytes + io, "unique_pairs": uniq,
+            "summary": s_bytes, "chunks": chunk_bytes}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_sample(wl, n_rows: int, seed: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload: all summaries + n rows."""
+    from threadpoolctl import threadpool_limits
+    from oracle import rdl_oracle as O
+    from diffusion_lms_b200.workloads import as_f64
+    f = {n: as_f64(getattr(wl, n)) for n in ("q", "q_mask", "k", "v", "x", "w_down", "w_up")}
+    dm = wl.dims
+    rng = np.random.default_rng(seed)
+    pos = np.arange(dm.L) if wl.q_pos is None else wl.q_pos[0]
+    cand = np.array([i for i in range(dm.Lq) if pos[i] % 64 != 63])
+    rows = np.sort(rng.choice(cand, size=min(n_rows, cand.size), replace=False))
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        s, H, _ = O.summary_pool(f["q_mask"], f["k"], f["v"])
+        idx, z = O.route_score_topk(f["q"], wl.q_pos, f["x"], f["w_down"], f["w_up"], s, H,
+                                    Hkv=dm.Hkv, K=dm.K, w=dm.w, lam=dm.lam, L=dm.L, rows=rows)
+        O.route_attn(f["q"], wl.q_pos, f["k"], f["v"], idx, z, w=dm.w, rows=rows)
+        dt = time.perf_counter() - t0
+    return dt, rows.size
+
+
+def run_reference(args, rank):
+    from diffusion_lms_b200 import workloads as W
+    if rank != 0:
+        return
+    wl = W.prefill_16k()
+    n = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(wl, max(1, n // 8))
+    times = [oracle_sample(wl, n, seed=s)[0] for s in range(args.steps)]
+    ms = 1e3 * statistics.mean(times)
+    val = n / (ms / 1e3)
+    sample = (f"all 256x28 summaries + {n} random content rows of the 16K prefill per step "
+              f"(fp64 NumPy, 1 BLAS thread)")
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "L": 16384, "Hq": 28, "Hkv": 4, "d": 128, "K": 32,
+                       "w": 256, "r": 64, "D": 3584, "rows_per_step": n},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=96)
+    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=dev)
+
+    from diffusion_lms_b200 import api, rdl
+    from diffusion_lms_b200 import workloads as W
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    # ---------------- 16K prefill route layer (the headline workload)
+    wl = W.prefill_16k(seed=2 + 1000 * rank)
+    inp = api.to_device(wl, dev)
+    out = api.alloc_outputs(inp.dims, inp.dtype, dev)
+
+    def step():
+        api.route_layer(inp, out, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert rdl.rdl_last_device_status() == rdl.OK
+
+    n_evt = 4
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_evt)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = rdl.launch_count()
+    for s_ in range(args.steps):
+        flush.zero_()                       # L2 flushed between timed steps (not timed)
+        e = ev[s_]
+        e[0].record(stream)
+        api.summary_pool(inp, out, stream=stream)
+        e[1].record(stream)
+        api.score_topk(inp, out, stream=stream)
+        e[2].record(stream)
+        api.route_attn(inp, out, stream=stream)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    launches = rdl.launch_count() - launches0
+    barrier()
+    clk = clocks.stop()
+    per = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_evt - 1)] for e in ev])
+    ms_step_local = float(per.sum(axis=1).mean())
+    ms_step = max_over_ranks(ms_step_local)
+    content_rows = int(((np.arange(wl.dims.L) % 64) != 63).sum())
+    value = world * content_rows / (ms_step / 1e3)
+    call_ms = per.mean(axis=0)
+    assert rdl.rdl_last_device_status() == rdl.OK
+
+    idx_np = out.idx.cpu().numpy()
+    fl_attn = attn_flops(wl.dims, None, idx_np)
+    fl_score = score_flops(wl.dims)
+    pk, pk_kind = peaks()
+    calls = {"rdl_summary_pool": float(call_ms[0]), "rdl_route_score_topk": float(call_ms[1]),
+             "rdl_route_attn": float(call_ms[2])}
+    dominant = max(calls, key=calls.get)
+    if dominant == "rdl_route_attn":
+        achieved = fl_attn / (call_ms[2] / 1e3) / 1e12
+        roof = {"kernel": "rdl_route_attn (window + chunk launches)", "bound": "tensor",
+                "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "algorithmic_flops": fl_attn, "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
+    elif dominant == "rdl_route_score_topk":
+        achieved = fl_score / (call_ms[1] / 1e3) / 1e12
+        roof = {"kernel": "rdl_route_score_topk", "bound": "tensor", "achieved": achieved,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "traffic": None, "algorithmic_flops": fl_score,
+                "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
+    else:
+        by = 2 * 2 * wl.dims.Hkv * wl.dims.L * wl.dims.d + 4 * wl.dims.Hq * (wl.dims.L // 64) * (wl.dims.d + 1)
+        achieved = by / (call_ms[0] / 1e3) / 1e9
+        roof = {"kernel": "rdl_summary_pool", "bound": "hbm", "achieved": achieved,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": None, "peak_source": f"hbm_gbs ({pk_kind})"}
+
+    # ---------------- end to end through the public API with host buffers
+    pin = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "x", "w_down", "w_up")}
+    h_o = torch.empty_like(out.o, device="cpu").pin_memory()
+    h_idx = torch.empty_like(out.idx, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = h_o.numel() * h_o.element_size() + h_idx.numel() * h_idx.element_size()
+
+    def e2e_step():
+        for n, t in pin.items():
+            getattr(inp, n).copy_(t, non_blocking=True)
+        api.route_layer(inp, out, stream=stream)
+        h_o.copy_(out.o, non_blocking=True)
+        h_idx.copy_(out.idx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+    e2e = {"value": world * content_rows / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del pin, h_o, h_idx
+
+    # ---------------- 128K decode block (summaries cached; score + attention)
+    decode = None
+    if not args.no_decode:
+        del inp, out
+        torch.cuda.empty_cache()
+        wd = W.decode_128k(seed=3 + 1000 * rank)
+        dinp = api.to_device(wd, dev)
+        dout = api.alloc_outputs(dinp.dims, dinp.dtype, dev)
+        api.summary_pool(dinp, dout, stream=stream)
+
+        def dstep():
+            api.score_topk(dinp, dout, stream=stream)
+            api.route_attn(dinp, dout, stream=stream)
+
+        for _ in range(args.warmup):
+            dstep()
+        torch.cuda.synchronize()
+        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        barrier()
+        for s_ in range(args.steps):
+            flush.zero_()
+            e = dev_ev[s_]
+            e[0].record(stream)
+            api.score_topk(dinp, dout, stream=stream)
+            e[1].record(stream)
+            api.route_attn(dinp, dout, stream=stream)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        dper = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in dev_ev])
+        d_ms = max_over_ranks(float(np.median(dper.sum(axis=1))))
+        db = decode_bytes(dinp.dims, dout.idx.cpu().numpy())
+        d_ach = db["total"] / (d_ms / 1e3) / 1e9
+        decode = {"workload": wd.name, "ms_per_step": d_ms,
+                  "score_ms": float(np.median(dper[:, 0])), "attn_ms": float(np.median(dper[:, 1])),
+                  "query_tokens_per_s": world * 32 / (d_ms / 1e3),
+                  "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                               "frac": d_ach / pk["hbm_gbs"], "algorithmic_bytes": db["total"],
+                               "unique_group_chunk_pairs": db["unique_pairs"],
+                               "peak_source": f"hbm_gbs ({pk_kind})"}}
+        assert rdl.rdl_last_device_status() == rdl.OK
+
+    # ---------------- CPU baseline (rank 0, oracle on a bounded sample)
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, n = oracle_sample(wl, args.cpu_rows)
+        cpu = {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"all 256x28 summaries + {n} random content rows of the 16K prefill "
+                         f"(fp64 NumPy, 1 BLAS thread), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "L": 16384, "Hq": 28, "Hkv": 4, "d": 128, "K": 32,
+                           "w": 256, "r": 64, "D": 3584, "content_rows": content_rows,
+                           "l2": "flushed between timed steps (256 MB write, untimed)",
+                           "parallelism": f"independent sequence per GPU x{world}"},
+                "breakdown_ms": calls, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk, "decode_128k": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,343 @@
+// C ABI of librdl.so (declared in include/rdl.h): argument checks on the host, workspace
+// layout and kernel dispatch.  Nothing here allocates, frees or synchronises (apart from
+// rdl_last_device_status, which is documented to synchronise).
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstdio>
+
+#include "common.cuh"
+#include "summary_pool.cuh"
+#include "score.cuh"
+#include "window_attn.cuh"
+#include "chunk_attn.cuh"
+
+using namespace rdl;
+
+namespace rdl {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace rdl
+
+namespace {
+
+constexpr int kMaxK = 64;
+constexpr int kMaxR = 128;
+constexpr int kMaxC = 8192;        // top-K keeps a whole score row per warp in shared memory
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool dims_ok(const rdl_dims* dm) {
+  if (!dm) return false;
+  if (dm->B < 1 || dm->L < S || dm->L % S != 0 || dm->Lq < 1) return false;
+  if (dm->Hq < 1 || dm->Hkv < 1 || dm->Hq % dm->Hkv != 0) return false;
+  if (dm->d != 64 && dm->d != 128) return false;
+  const long long rows = (long long)dm->B * dm->Lq * dm->Hq * dm->d;
+  const long long kv = (long long)dm->B * dm->Hkv * dm->L * dm->d;
+  if (rows > (1LL << 40) || kv > (1LL << 40)) return false;
+  return true;
+}
+bool dtype_ok(rdl_dtype t) { return t == RDL_BF16 || t == RDL_F32; }
+bool route_dims_ok(const rdl_dims* dm) {
+  if (!dims_ok(dm)) return false;
+  const int C = dm->L / S;
+  if (dm->K < 1 || dm->K > kMaxK || dm->K > C) return false;
+  if (dm->r < 0 || dm->r > kMaxR) return false;
+  if (dm->r > 0 && dm->D < 1) return false;
+  return true;
+}
+// bf16, head dim 128 and at most 8 heads per group run on the tensor-core kernels;
+// everything else on the scalar kernels.
+bool fast_attn(const rdl_dims* dm, rdl_dtype t) {
+  return t == RDL_BF16 && dm->d == 128 && dm->Hq / dm->Hkv <= 8;
+}
+int attn_splits(const rdl_dims* dm) {
+  const long long items = (long long)dm->B * dm->Lq * dm->Hkv;
+  if (items >= 4096) return 1;
+  int ns = (int)((4096 + items - 1) / items);
+  return ns < 8 ? (ns < dm->K ? ns : dm->K) : (8 < dm->K ? 8 : dm->K);
+}
+
+struct ScoreWs {
+  size_t t, qres, z_all, zeta, total;
+};
+ScoreWs score_ws(const rdl_dims* dm) {
+  const size_t C = dm->L / S;
+  ScoreWs w{};
+  size_t off = 0;
+  w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
+  w.qres = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * dm->Hq * dm->d);
+  w.z_all = off; off += align256(sizeof(float) * (size_t)dm->B * dm->Hq * dm->Lq * C);
+  w.zeta = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
+  w.total = off;
+  return w;
+}
+struct AttnWs {
+  size_t o_loc, lam_loc, o_acc, total;
+};
+AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
+  AttnWs w{};
+  if (!fast_attn(dm, t)) return w;
+  const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
+  size_t off = 0;
+  w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d);
+  w.lam_loc = off; off += align256(sizeof(float) * rows);
+  w.o_acc = off;
+  const int ns = attn_splits(dm);
+  if (ns > 1) off += align256(sizeof(float) * rows * dm->d * ns);
+  w.total = off;
+  return w;
+}
+
+rdl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RDL_OK : RDL_ERR_CUDA; }
+
+// |p - j| <= w with p, j in [0, L) never exceeds L - 1, so a radius >= L means "everything"
+// and any negative radius means "no window"; clamping keeps device index math in range.
+rdl_dims clamp_w(const rdl_dims* d) {
+  rdl_dims c = *d;
+  if (c.w > c.L) c.w = c.L;
+  if (c.w < 0) c.w = -1;
+  return c;
+}
+
+template <typename T>
+rdl_status score_impl(const void* q, const int32_t* q_pos, const void* x, const void* w_down,
+                      const void* w_up, const float* summary, const float* entropy,
+                      const rdl_dims* dm, int32_t* idx, float* z_sel, void* workspace,
+                      cudaStream_t st) {
+  const ScoreWs wl = score_ws(dm);
+  char* ws = static_cast<char*>(workspace);
+  float* t = reinterpret_cast<float*>(ws + wl.t);
+  float* qres = reinterpret_cast<float*>(ws + wl.qres);
+  float* z_all = reinterpret_cast<float*>(ws + wl.z_all);
+  float* zeta = reinterpret_cast<float*>(ws + wl.zeta);
+  const int M = dm->B * dm->Lq, N = dm->Hq * dm->d, C = dm->L / S;
+  const T* qT = static_cast<const T*>(q);
+  if (dm->r > 0 && x) {
+    dim3 g1((dm->r + 63) / 64, (M + 63) / 64);
+    count_launch(2);
+    gemm_f32_kernel<T, T, T><<<g1, 256, 0, st>>>(static_cast<const T*>(x), static_cast<const T*>(w_down),
+                                                 (const T*)nullptr, t, M, dm->r, dm->D);
+    dim3 g2((N + 63) / 64, (M + 63) / 64);
+    gemm_f32_kernel<float, T, T><<<g2, 256, 0, st>>>(t, static_cast<const T*>(w_up), qT, qres, M, N, dm->r);
+  } else {
+    // no residual: q_res = q (an r = 0 product adds nothing)
+    count_launch();
+    dim3 g2((N + 63) / 64, (M + 63) / 64);
+    gemm_f32_kernel<float, T, T><<<g2, 256, 0, st>>>(t, static_cast<const T*>(w_up), qT, qres, M, N, 0);
+  }
+  dim3 g3((C + 63) / 64, (dm->Lq + 63) / 64, dm->B * dm->Hkv);
+  count_launch(2);   // zeta + top-K
+  if (dm->d == 128)
+    zeta_kernel<128><<<g3, 256, 0, st>>>(qres, q_pos, summary, entropy, dm->Lq, dm->L, dm->Hq, dm->Hkv,
+                                         dm->w, dm->lambda, z_all, zeta);
+  else
+    zeta_kernel<64><<<g3, 256, 0, st>>>(qres, q_pos, summary, entropy, dm->Lq, dm->L, dm->Hq, dm->Hkv,
+                                        dm->w, dm->lambda, z_all, zeta);
+  const int warps = 4;
+  const size_t smem = (size_t)warps * C * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return RDL_ERR_CUDA;
+  dim3 g4((unsigned)(((long long)dm->Lq * dm->Hkv + warps - 1) / warps), dm->B);
+  topk_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
+                                            idx, z_sel);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T, bool ROUTE>
+rdl_status generic_attn(const void* q, const int32_t* q_pos, const void* k, const void* v,
+                        const int32_t* idx, const float* z_sel, const rdl_dims* dm, void* o,
+                        float* lse, cudaStream_t st) {
+  dim3 grid(dm->Lq, dm->Hkv, dm->B);
+  count_launch();
+  const T *qT = static_cast<const T*>(q), *kT = static_cast<const T*>(k), *vT = static_cast<const T*>(v);
+  if (dm->d == 128)
+    generic_attn_kernel<T, 128, ROUTE><<<grid, 128, 0, st>>>(qT, q_pos, kT, vT, idx, z_sel, dm->L, dm->Lq,
+                                                            dm->Hq, dm->Hkv, dm->K, dm->w, dm->flags,
+                                                            static_cast<T*>(o), lse);
+  else
+    generic_attn_kernel<T, 64, ROUTE><<<grid, 128, 0, st>>>(qT, q_pos, kT, vT, idx, z_sel, dm->L, dm->Lq,
+                                                           dm->Hq, dm->Hkv, dm->K, dm->w, dm->flags,
+                                                           static_cast<T*>(o), lse);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int MODE>
+rdl_status launch_window_mma(const void* q, const int32_t* q_pos, const void* k, const void* v,
+                             const rdl_dims* dm, void* o, float* lse, float* o_loc, float* lam_loc,
+                             cudaStream_t st) {
+  const int G = dm->Hq / dm->Hkv;
+  const size_t smem = window_mma_smem(G);
+  auto kern = window_mma_kernel<MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  dim3 grid((dm->Lq + WIN_ROWS - 1) / WIN_ROWS, dm->B * dm->Hkv);
+  count_launch();
+  kern<<<grid, 32 * G, smem, st>>>(static_cast<const __nv_bfloat16*>(q), q_pos,
+                                   static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                                   dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->w, static_cast<__nv_bfloat16*>(o), lse,
+                                   o_loc, lam_loc);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rdl_version(void) { return "0.1.0"; }
+
+unsigned long long rdl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* rdl_status_string(rdl_status s) {
+  switch (s) {
+    case RDL_OK: return "ok";
+    case RDL_ERR_INVALID_ARG: return "invalid argument";
+    case RDL_ERR_UNSUPPORTED: return "unsupported combination";
+    case RDL_ERR_CUDA: return "CUDA error";
+    case RDL_ERR_TIMEOUT: return "device wait timed out";
+    case RDL_ERR_WORKSPACE: return "workspace too small";
+    case RDL_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+size_t rdl_workspace_bytes(int which, const rdl_dims* dims, rdl_dtype dtype) {
+  if (!route_dims_ok(dims) || !dtype_ok(dtype)) return 0;
+  if (which == RDL_WS_SCORE) return score_ws(dims).total;
+  if (which == RDL_WS_ATTN) return attn_ws(dims, dtype).total;
+  return 0;
+}
+
+rdl_status rdl_summary_pool(const void* q_mask, long long q_chunk_stride, long long q_batch_stride,
+                            const void* k, const void* v, const rdl_dims* dims, rdl_dtype dtype,
+                            float* summary, float* entropy, void* o_mask, void* stream) {
+  if (!dims_ok(dims) || !dtype_ok(dtype)) return RDL_ERR_INVALID_ARG;
+  if (!q_mask || !k || !summary || !entropy) return RDL_ERR_INVALID_ARG;
+  if (o_mask && !v) return RDL_ERR_INVALID_ARG;
+  if (!aligned16(q_mask) || !aligned16(k) || (v && !aligned16(v)) || !aligned16(summary) ||
+      (o_mask && !aligned16(o_mask)))
+    return RDL_ERR_INVALID_ARG;
+  const long long row = (long long)dims->Hq * dims->d;
+  if (q_chunk_stride < row || q_batch_stride < 0) return RDL_ERR_INVALID_ARG;
+  const cudaStream_t st = as_stream(stream);
+  cudaError_t e;
+  if (dtype == RDL_BF16) {
+    e = dims->d == 128 ? launch_summary_pool<__nv_bfloat16, 128>(q_mask, q_chunk_stride, q_batch_stride, k, v,
+                                                                 *dims, summary, entropy, o_mask, st)
+                       : launch_summary_pool<__nv_bfloat16, 64>(q_mask, q_chunk_stride, q_batch_stride, k, v,
+                                                                *dims, summary, entropy, o_mask, st);
+  } else {
+    e = dims->d == 128 ? launch_summary_pool<float, 128>(q_mask, q_chunk_stride, q_batch_stride, k, v, *dims,
+                                                         summary, entropy, o_mask, st)
+                       : launch_summary_pool<float, 64>(q_mask, q_chunk_stride, q_batch_stride, k, v, *dims,
+                                                        summary, entropy, o_mask, st);
+  }
+  return cuda_status(e);
+}
+
+rdl_status rdl_route_score_topk(const void* q, const int32_t* q_pos, const void* x,
+                                const void* w_down, const void* w_up, const float* summary,
+                                const float* entropy, const rdl_dims* dims, rdl_dtype dtype,
+                                int32_t* idx, float* z_sel, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  if (!route_dims_ok(dims) || !dtype_ok(dtype)) return RDL_ERR_INVALID_ARG;
+  if (!q_pos && dims->Lq != dims->L) return RDL_ERR_INVALID_ARG;
+  if (dims->L / S > kMaxC) return RDL_ERR_UNSUPPORTED;
+  const bool residual = dims->r > 0 && x != nullptr;
+  if (!q || !summary || !entropy || !idx || !z_sel || !workspace) return RDL_ERR_INVALID_ARG;
+  if (residual && (!w_down || !w_up)) return RDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summary) || !aligned16(entropy) || !aligned16(idx) ||
+      !aligned16(z_sel) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (residual && (!aligned16(x) || !aligned16(w_down) || !aligned16(w_up))) ||
+      (q_pos && !aligned16(q_pos)))
+    return RDL_ERR_INVALID_ARG;
+  if (ws_bytes < score_ws(dims).total) return RDL_ERR_WORKSPACE;
+  rdl_dims dm = clamp_w(dims);
+  if (!residual) dm.r = 0;
+  const cudaStream_t st = as_stream(stream);
+  return dtype == RDL_BF16 ? score_impl<__nv_bfloat16>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx,
+                                                       z_sel, workspace, st)
+                           : score_impl<float>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel,
+                                               workspace, st);
+}
+
+rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, const void* v,
+                          const int32_t* idx, const float* z_sel, const rdl_dims* dims,
+                          rdl_dtype dtype, void* o, float* lse, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  if (!route_dims_ok(dims) || !dtype_ok(dtype)) return RDL_ERR_INVALID_ARG;
+  if (!q_pos && dims->Lq != dims->L) return RDL_ERR_INVALID_ARG;
+  if (!q || !k || !v || !idx || !z_sel || !o) return RDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(z_sel) ||
+      !aligned16(o) || (lse && !aligned16(lse)) || (q_pos && !aligned16(q_pos)))
+    return RDL_ERR_INVALID_ARG;
+  const cudaStream_t st = as_stream(stream);
+  const rdl_dims dmc = clamp_w(dims);
+  dims = &dmc;
+  if (!fast_attn(dims, dtype)) {
+    return dtype == RDL_BF16 ? generic_attn<__nv_bfloat16, true>(q, q_pos, k, v, idx, z_sel, dims, o, lse, st)
+                             : generic_attn<float, true>(q, q_pos, k, v, idx, z_sel, dims, o, lse, st);
+  }
+  const AttnWs wl = attn_ws(dims, dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RDL_ERR_INVALID_ARG;
+  if (ws_bytes < wl.total) return RDL_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  float* o_loc = reinterpret_cast<float*>(ws + wl.o_loc);
+  float* lam_loc = reinterpret_cast<float*>(ws + wl.lam_loc);
+  float* o_acc = reinterpret_cast<float*>(ws + wl.o_acc);
+  rdl_status s = launch_window_mma<1>(q, q_pos, k, v, dims, nullptr, nullptr, o_loc, lam_loc, st);
+  if (s != RDL_OK) return s;
+  const int ns = attn_splits(dims);
+  const size_t rows = (size_t)dims->B * dims->Lq * dims->Hq;
+  const size_t smem = (size_t)CH_WARPS * CH_WARP_SMEM;
+  if (cudaFuncSetAttribute(chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return RDL_ERR_CUDA;
+  const long long warps = (long long)dims->Lq * dims->Hkv * ns;
+  dim3 grid((unsigned)((warps + CH_WARPS - 1) / CH_WARPS), dims->B);
+  count_launch(ns > 1 ? 2 : 1);
+  chunk_mma_kernel<<<grid, CH_WARPS * 32, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(q), q_pos, static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), idx, z_sel, o_loc, lam_loc, dims->L, dims->Lq, dims->Hq, dims->Hkv,
+      dims->K, dims->w, ns, dims->flags, static_cast<__nv_bfloat16*>(o), lse, o_acc);
+  if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+  if (ns > 1) {
+    const long long n = (long long)rows * dims->d;
+    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    chunk_finalize_kernel<<<blocks, 256, 0, st>>>(o_acc, ns, q_pos, dims->Lq, dims->Hq * dims->d, dims->B,
+                                                  static_cast<__nv_bfloat16*>(o));
+    if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+  }
+  return RDL_OK;
+}
+
+rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, const void* v,
+                        const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse, void* stream) {
+  if (!dims_ok(dims) || !dtype_ok(dtype) || dims->w < 0) return RDL_ERR_INVALID_ARG;
+  if (!q_pos && dims->Lq != dims->L) return RDL_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o) return RDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      (q_pos && !aligned16(q_pos)))
+    return RDL_ERR_INVALID_ARG;
+  const cudaStream_t st = as_stream(stream);
+  const rdl_dims dmc = clamp_w(dims);
+  dims = &dmc;
+  if (!fast_attn(dims, dtype)) {
+    return dtype == RDL_BF16 ? generic_attn<__nv_bfloat16, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st)
+                             : generic_attn<float, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st);
+  }
+  return launch_window_mma<0>(q, q_pos, k, v, dims, o, lse, nullptr, nullptr, st);
+}
+
+rdl_status rdl_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return RDL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return RDL_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return RDL_ERR_CUDA;
+  return static_cast<rdl_status>(v);
+}
+
+}  // extern "C"

@@ -78,9 +78,19 @@ class Workload:
 def bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 to bfloat16 (round to nearest, ties to even); returns uint16 bits."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    b = x.view(np.uint32)
-    bias = ((b >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
-    return ((b + bias) >> np.uint32(16)).astype(np.uint16)
+    flat = x.reshape(-1).view(np.uint32)
+    out = np.empty(flat.size, dtype=np.uint16)
+    t = np.empty(min(flat.size, _BLOCK), dtype=np.uint32)
+    for s in range(0, flat.size, _BLOCK):
+        e = min(flat.size, s + _BLOCK)
+        b, tt = flat[s:e], t[:e - s]
+        np.right_shift(b, 16, out=tt)
+        np.bitwise_and(tt, 1, out=tt)
+        tt += np.uint32(0x7FFF)
+        tt += b
+        tt >>= np.uint32(16)
+        out[s:e] = tt
+    return out.reshape(x.shape)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -171,14 +181,18 @@ def make_inputs(dims: Dims, *, seed: int, n_needles: int = 0, unit_scale: bool =
     if n_needles:
         needles = np.stack([np.sort(rng.choice(C, size=n_needles, replace=False))
                             for _ in range(B)])
-        qf = as_f64(q)                                                     # [B,Lq,Hq,d]
-        if q_pos is None:
-            content = (np.arange(L) % CHUNK) != CHUNK - 1
-            qf = qf[:, content]
         knorm = 1.0 if unit_scale else float(np.sqrt(d))
         for b in range(B):
+            qb = bf16_to_f32(q[b]) if q.dtype == np.uint16 else q[b]        # [Lq,Hq,d] exact
             for g in range(Hkv):
-                u = qf[b, :, g * G:(g + 1) * G, :].reshape(-1, d).mean(axis=0)
+                # mean raw query of the group over content rows (mask-slot rows excluded)
+                tot = qb[:, g * G:(g + 1) * G, :].sum(axis=(0, 1), dtype=np.float64)
+                n = qb.shape[0] * G
+                if q_pos is None:
+                    tot -= qb[CHUNK - 1::CHUNK, g * G:(g + 1) * G, :].sum(axis=(0, 1),
+                                                                           dtype=np.float64)
+                    n -= (qb.shape[0] // CHUNK) * G
+                u = tot / n
                 u /= np.linalg.norm(u)
                 shift = (0.5 * knorm * u).astype(np.float32)
                 for c in needles[b]:

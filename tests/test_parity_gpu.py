@@ -1,0 +1,210 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Small cases cover every row and span several tiles with ragged tails (C not a multiple
+of the 64-chunk score tile, Lq not a multiple of the 16-row window tile); the full-size
+workloads (16K / 64K prefill, 128K decode, 28-layer stack) are checked on sampled rows.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from diffusion_lms_b200 import api, rdl
+from diffusion_lms_b200 import workloads as W
+from oracle import rdl_oracle as O
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def small(**kw):
+    base = dict(B=1, L=2368, Lq=2368, Hq=28, Hkv=4, d=128, D=512, r=64, K=8, w=100, lam=0.1,
+                dtype="bf16")
+    base.update(kw)
+    return W.Dims(**base)
+
+
+def test_tiny_f32_every_row():
+    wl = W.tiny_f32()
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(wl.dims.L)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_exact"] > 0
+    P.check_swa(wl, gpu, rows)
+
+
+def test_bf16_prefill_ragged_every_row():
+    wl = W.make_inputs(small(), seed=11, n_needles=4)
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(wl.dims.L)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_exact"] > 1000
+    P.check_swa(wl, gpu, rows)
+
+
+def test_bf16_decode_block_split_path():
+    dm = small(L=8192, Lq=32, K=32, w=256)
+    wl = W.make_inputs(dm, seed=12, n_needles=8, decode_block=32)
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(32)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+def test_bf16_scattered_positions_ragged_rows():
+    """37 rows at arbitrary positions (mask slots, both ends), not a multiple of 16."""
+    dm = small(L=4096, Lq=37, K=8, w=100)
+    wl = W.make_inputs(dm, seed=13, n_needles=4, decode_block=37)
+    rng = np.random.default_rng(5)
+    pos = np.concatenate([[0, 1, 63, 64, 127, 4095, 4094, 4032], rng.integers(0, 4096, 29)])
+    wl.q_pos = pos.astype(np.int32)[None, :]
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(37)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (2, 2), (6, 1)])
+def test_group_sizes(Hq, Hkv):
+    wl = W.make_inputs(small(L=1024, Lq=1024, Hq=Hq, Hkv=Hkv, K=6, w=70), seed=14, n_needles=2)
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(1024)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+def test_bf16_head_dim_64_batch_2():
+    wl = W.make_inputs(small(B=2, L=1024, Lq=1024, Hq=8, Hkv=2, d=64, K=4, w=64), seed=15,
+                       n_needles=2)
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(0, 1024, 3)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+@pytest.mark.parametrize("case", ["no_window", "window_covers_all", "lambda0_no_residual",
+                                  "mean_summary", "K_equals_C"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_edge_cases(case, dtype):
+    kw = dict(L=1024, Lq=1024, Hq=8, Hkv=2, K=4, w=64, dtype=dtype)
+    flags, with_res, mean = 0, True, False
+    if case == "no_window":
+        kw["w"] = -1
+    elif case == "window_covers_all":
+        kw["w"] = 5000
+    elif case == "lambda0_no_residual":
+        kw["lam"] = 0.0
+        with_res = False
+    elif case == "mean_summary":
+        flags, mean = rdl.FLAG_MEAN_SUMMARY, True
+    elif case == "K_equals_C":
+        kw.update(K=16, w=10)
+    wl = W.make_inputs(small(**kw), seed=16, n_needles=2, unit_scale=(dtype == "f32"))
+    gpu = P.run_gpu(wl, flags=flags, with_residual=with_res, swa=kw["w"] >= 0)
+    rows = np.arange(1024)
+    P.check_route_layer(wl, gpu, rows, mean_summary=mean, with_residual=with_res)
+    if kw["w"] >= 0:
+        P.check_swa(wl, gpu, rows)
+
+
+def test_device_checks_record_without_fault():
+    """Out-of-range and in-window chunk ids are recorded in the status word and skipped."""
+    wl = W.make_inputs(small(L=1024, Lq=1024, Hq=8, Hkv=2, K=4, w=64), seed=17)
+    inp = api.to_device(wl)
+    inp.dims.flags = rdl.FLAG_CHECKS
+    out = api.alloc_outputs(inp.dims, inp.dtype)
+    api.summary_pool(inp, out)
+    api.score_topk(inp, out)
+    torch.cuda.synchronize()
+    assert rdl.rdl_last_device_status() == rdl.OK          # valid selection: no record
+    out.idx[0, 0, 500, 0] = 10_000                          # beyond C
+    out.idx[0, 1, 500, 1] = 500 // 64                       # the query's own chunk
+    api.route_attn(inp, out)
+    assert rdl.rdl_last_device_status() == rdl.ERR_DEVICE_CHECK
+    assert rdl.rdl_last_device_status() == rdl.OK          # cleared on read
+
+
+def test_bitwise_repeatable():
+    for dm, dec in ((small(), 0), (small(L=8192, Lq=32, K=32, w=256), 32)):
+        wl = W.make_inputs(dm, seed=18, n_needles=4, decode_block=dec)
+        a = P.run_gpu(wl, swa=True)
+        b = P.run_gpu(wl, swa=True)
+        for key in ("s", "H", "idx", "z", "o", "lse", "swa_o", "swa_lse"):
+            assert np.array_equal(a[key], b[key], equal_nan=True), key
+
+
+def test_head_permutation_and_locality():
+    wl = W.make_inputs(small(L=1024, Lq=1024, Hq=8, Hkv=2, K=3, w=64), seed=19, n_needles=2)
+    base = P.run_gpu(wl)
+    # permute the heads inside group 0 (queries, mask queries, residual columns)
+    perm = np.arange(8)
+    perm[:4] = perm[:4][::-1]
+    wl2 = dataclasses.replace(wl, q=wl.q[:, :, perm].copy(), q_mask=wl.q_mask[:, :, perm].copy(),
+                              w_up=wl.w_up.reshape(wl.w_up.shape[0], 8, -1)[:, perm]
+                              .reshape(wl.w_up.shape).copy())
+    per = P.run_gpu(wl2)
+    assert np.array_equal(per["idx"], base["idx"])
+    assert np.array_equal(per["o"][:, :, perm], base["o"])
+    # new values in chunks no row of group 0 selects or sees: group 0 outputs unchanged
+    i = 600
+    used = set(range(max(0, i - 64), i + 65))
+    for c in base["idx"][0, 0, i]:
+        used.update(range(64 * c, 64 * c + 64))
+    far = np.array([j for j in range(1024) if j not in used])
+    v2 = wl.v.copy()
+    v2[:, 0, far] = W.bf16_bits(np.random.default_rng(3).standard_normal(v2[:, 0, far].shape)
+                                .astype(np.float32))
+    mod = P.run_gpu(dataclasses.replace(wl, v=v2))
+    assert np.array_equal(mod["idx"], base["idx"])
+    assert np.array_equal(mod["o"][0, i, :4], base["o"][0, i, :4])
+
+
+# ----------------------------------------------------------------------------- full size
+
+@pytest.fixture(scope="module")
+def prefill16k():
+    return W.prefill_16k()
+
+
+def test_prefill_16k_sampled(prefill16k):
+    wl = prefill16k
+    gpu = P.run_gpu(wl, swa=True)
+    rows = P.sample_rows(wl, 512)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_exact"] > 1000
+    P.check_swa(wl, gpu, rows)
+    # properties that hold at any size, on every row
+    idx = gpu["idx"][0]
+    assert idx.shape == (4, 16384, 32) and idx.max() < 256
+    content = (np.arange(16384) % 64) != 63
+    assert np.all(idx[:, ~content] == -1) and np.all(idx[:, content] >= 0)
+    assert np.all(np.isfinite(gpu["o"])) and np.all(np.isfinite(gpu["lse"][:, :, content]))
+
+
+def test_decode_128k():
+    wl = W.decode_128k()
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(32)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+def test_prefill_64k_mixture_sampled():
+    wl = W.prefill_64k()
+    gpu = P.run_gpu(wl)
+    rows = P.sample_rows(wl, 512, seed=1)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_tie"] > 0          # the mixture keys create near ties
+
+
+def test_stack_128k_all_layers():
+    for layer in range(W.STACK_LAYERS):
+        wl = W.stack_layer(layer)
+        route = W.is_route_layer(layer)
+        gpu = P.run_gpu(wl, route=route, swa=not route)
+        rows = np.arange(32)
+        if route:
+            P.check_route_layer(wl, gpu, rows)
+        else:
+            P.check_swa(wl, gpu, rows)
