@@ -199,6 +199,7 @@ const char* rdl_status_string(rdl_status s) {
     case RDL_ERR_TIMEOUT: return "device wait timed out";
     case RDL_ERR_WORKSPACE: return "workspace too small";
     case RDL_ERR_DEVICE_CHECK: return "device-side check failed";
+    case RDL_ERR_SCRATCH_LIMIT: return "size exceeds the static scratch of the no-allocation entry point";
   }
   return "unknown status";
 }
@@ -341,3 +342,45 @@ rdl_status rdl_last_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// rdl_route_attn_noalloc: rdl_route_attn with a library-held static scratch array, for
+// hosts that cannot hand the library device memory at call time (engines that plan all
+// device buffers before serving, plugin interfaces without an allocator).  It forwards to
+// rdl_route_attn with the array as the workspace; no allocation anywhere on this path.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = RDL_NOALLOC_SCRATCH_BYTES;
+// One copy per device that loads the library, held until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address must come from cudaGetSymbolAddress,
+// looked up once per device with that device current (the first call on that device).
+void* noalloc_scratch_ptr() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  return p;
+}
+
+}  // namespace
+
+extern "C" rdl_status rdl_route_attn_noalloc(const void* q, const int32_t* q_pos, const void* k,
+                                             const void* v, const int32_t* idx, const float* z_sel,
+                                             const rdl_dims* dims, rdl_dtype dtype, void* o,
+                                             float* lse, void* stream) {
+  if (!route_dims_ok(dims) || !dtype_ok(dtype)) return RDL_ERR_INVALID_ARG;
+  const rdl_dims dmc = clamp_w(dims);
+  if (attn_ws(&dmc, dtype).total > kNoAllocScratchBytes) return RDL_ERR_SCRATCH_LIMIT;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return RDL_ERR_CUDA;
+  return rdl_route_attn(q, q_pos, k, v, idx, z_sel, dims, dtype, o, lse, scratch,
+                        kNoAllocScratchBytes, stream);
+}

@@ -23,6 +23,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_DEVICE_CHECK = \
     0, -1, -2, -3, -4, -5, -6
+ERR_SCRATCH_LIMIT = -7
+NOALLOC_SCRATCH_BYTES = 16 << 20
 BF16, F32 = 0, 1
 FLAG_MEAN_SUMMARY, FLAG_CHECKS = 0x1, 0x2
 WS_SCORE, WS_ATTN = 0, 1
@@ -49,6 +51,7 @@ _SIGS = {
     "rdl_route_score_topk": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp,
                                     _sz, _vp]),
     "rdl_route_attn": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp, _sz, _vp]),
+    "rdl_route_attn_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp]),
     "rdl_swa_attn": (_int, [_vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp]),
     "rdl_workspace_bytes": (_sz, [_int, _P, _int]),
     "rdl_last_device_status": (_int, [_vp]),
@@ -167,6 +170,16 @@ def rdl_route_attn(q, q_pos, k, v, idx, z_sel, dims: Dims, dtype, o, lse=None, w
                             ctypes.byref(dims.c()), _dt(dtype), _p(o), _p(lse), _p(workspace),
                             ws_bytes, _stream(stream))
     return _check("rdl_route_attn", s, raise_on_error)
+
+
+def rdl_route_attn_noalloc(q, q_pos, k, v, idx, z_sel, dims: Dims, dtype, o, lse=None,
+                           stream=None, raise_on_error=True) -> int:
+    """rdl_route_attn without a workspace argument: for hosts that cannot allocate device
+    memory at call time; librdl uses its own static device scratch (16 MiB per device)."""
+    s = _lib.rdl_route_attn_noalloc(_p(q), _p(q_pos), _p(k), _p(v), _p(idx), _p(z_sel),
+                                    ctypes.byref(dims.c()), _dt(dtype), _p(o), _p(lse),
+                                    _stream(stream))
+    return _check("rdl_route_attn_noalloc", s, raise_on_error)
 
 
 def rdl_swa_attn(q, q_pos, k, v, dims: Dims, dtype, o, lse=None, stream=None,

@@ -56,7 +56,8 @@ typedef enum {
   RDL_ERR_CUDA = -3,
   RDL_ERR_TIMEOUT = -4,
   RDL_ERR_WORKSPACE = -5,
-  RDL_ERR_DEVICE_CHECK = -6
+  RDL_ERR_DEVICE_CHECK = -6,
+  RDL_ERR_SCRATCH_LIMIT = -7
 } rdl_status;
 
 typedef enum { RDL_BF16 = 0, RDL_F32 = 1 } rdl_dtype;
@@ -151,6 +152,33 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
                           const int32_t* idx, const float* z_sel, const rdl_dims* dims,
                           rdl_dtype dtype, void* o, float* lse, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/*
+ * rdl_route_attn_noalloc -- rdl_route_attn for callers that cannot allocate device memory.
+ * The paper has no counterpart to this call: it exists for deployment.  Some hosts give a
+ * kernel library no way to obtain scratch memory at call time -- inference engines that
+ * plan every device buffer before serving and forbid allocation on the request path (a
+ * cudaMalloc there synchronises the device and can fail once memory is fragmented), and
+ * plugin interfaces that hand the plugin its inputs and outputs but no allocator.  This
+ * entry point takes the same arguments as rdl_route_attn minus the workspace and uses a
+ * static scratch array that librdl.so itself holds in device memory instead.
+ *
+ * Scratch limit: RDL_NOALLOC_SCRATCH_BYTES (16 MiB) per device, reserved on every GPU
+ * that loads the library, until the process exits.  A call whose
+ * rdl_workspace_bytes(RDL_WS_ATTN, dims, dtype) exceeds it returns RDL_ERR_SCRATCH_LIMIT
+ * and launches nothing (a 32-query decode block over 28 heads needs about 4.2 MiB).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture begins.
+ * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ * Every call on a device shares the one array and leaves its contents behind; no part of
+ * it needs to start at zero.  Calls that overlap on the GPU (concurrent streams, or
+ * several host threads) race on the array: serialise them.
+ */
+#define RDL_NOALLOC_SCRATCH_BYTES (16u << 20)
+rdl_status rdl_route_attn_noalloc(const void* q, const int32_t* q_pos, const void* k,
+                                  const void* v, const int32_t* idx, const float* z_sel,
+                                  const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse,
+                                  void* stream);
 
 /*
  * rdl_swa_attn -- bidirectional sliding-window attention of the non-route layers
