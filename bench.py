@@ -135,6 +135,29 @@ def decode_bytes(dims, idx) -> dict:
             "summary": s_bytes, "chunks": chunk_bytes}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent sequence (no data exchange between ranks)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank time over all ranks (every rank calls it the same number of times)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(rows_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job rows per second: all ranks' rows over the slowest rank's time."""
+    return world * rows_per_rank / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- oracle arm
 
 def oracle_sample(wl, n_rows: int, seed: int = 0):
@@ -222,18 +245,14 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
     # ---------------- 16K prefill route layer (the headline workload)
-    wl = W.prefill_16k(seed=2 + 1000 * rank)
+    wl = W.prefill_16k(seed=rank_seed(2, rank))
     inp = api.to_device(wl, dev)
     out = api.alloc_outputs(inp.dims, inp.dtype, dev)
 
@@ -269,9 +288,9 @@ def main():
     clk = clocks.stop()
     per = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_evt - 1)] for e in ev])
     ms_step_local = float(per.sum(axis=1).mean())
-    ms_step = max_over_ranks(ms_step_local)
+    ms_step = max_ranks(ms_step_local)
     content_rows = int(((np.arange(wl.dims.L) % 64) != 63).sum())
-    value = world * content_rows / (ms_step / 1e3)
+    value = job_throughput(content_rows, world, ms_step)
     call_ms = per.mean(axis=0)
     assert rdl.rdl_last_device_status() == rdl.OK
 
@@ -326,8 +345,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
-    e2e = {"value": world * content_rows / (e2e_ms / 1e3), "unit": UNIT,
+    e2e_ms = max_ranks(e0.elapsed_time(e1) / n_e2e)
+    e2e = {"value": job_throughput(content_rows, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     del pin, h_o, h_idx
 
@@ -336,7 +355,7 @@ def main():
     if not args.no_decode:
         del inp, out
         torch.cuda.empty_cache()
-        wd = W.decode_128k(seed=3 + 1000 * rank)
+        wd = W.decode_128k(seed=rank_seed(3, rank))
         dinp = api.to_device(wd, dev)
         dout = api.alloc_outputs(dinp.dims, dinp.dtype, dev)
         api.summary_pool(dinp, dout, stream=stream)
@@ -360,7 +379,7 @@ def main():
             e[2].record(stream)
         torch.cuda.synchronize()
         dper = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in dev_ev])
-        d_ms = max_over_ranks(float(np.median(dper.sum(axis=1))))
+        d_ms = max_ranks(float(np.median(dper.sum(axis=1))))
         db = decode_bytes(dinp.dims, dout.idx.cpu().numpy())
         d_ach = db["total"] / (d_ms / 1e3) / 1e9
         decode = {"workload": wd.name, "ms_per_step": d_ms,

@@ -2,6 +2,7 @@
 // layout and kernel dispatch.  Nothing here allocates, frees or synchronises (apart from
 // rdl_last_device_status, which is documented to synchronise).
 #include <atomic>
+#include <type_traits>
 #include <climits>
 #include <cstdint>
 #include <cstdio>
@@ -9,6 +10,7 @@
 #include "common.cuh"
 #include "summary_pool.cuh"
 #include "score.cuh"
+#include "score_mma.cuh"
 #include "window_attn.cuh"
 #include "chunk_attn.cuh"
 
@@ -60,17 +62,29 @@ int attn_splits(const rdl_dims* dm) {
   return ns < 8 ? (ns < dm->K ? ns : dm->K) : (8 < dm->K ? 8 : dm->K);
 }
 
+// The tensor-core score path: bf16, d = 128, rank 64 residual with D % 64 == 0, and
+// enough query rows to fill 128-row tiles.  Everything else runs the fp32 path.
+constexpr int kFastScoreMinRows = 128;
+bool fast_score(const rdl_dims* dm, rdl_dtype t) {
+  return t == RDL_BF16 && dm->d == 128 && dm->r == 64 && dm->D % 64 == 0 && dm->Hq / dm->Hkv <= 8 &&
+         dm->Lq >= kFastScoreMinRows;
+}
 struct ScoreWs {
-  size_t t, qres, z_all, zeta, total;
+  size_t t, qres, z_all, zeta, tt, sb, total;
 };
-ScoreWs score_ws(const rdl_dims* dm) {
+ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   const size_t C = dm->L / S;
   ScoreWs w{};
   size_t off = 0;
-  w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
-  w.qres = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * dm->Hq * dm->d);
   w.z_all = off; off += align256(sizeof(float) * (size_t)dm->B * dm->Hq * dm->Lq * C);
   w.zeta = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
+  if (fast_score(dm, dt)) {
+    w.tt = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Lq * 2 * dm->r);
+    w.sb = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Hq * C * (2 * dm->d + 2 * dm->r));
+  } else {
+    w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
+    w.qres = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * dm->Hq * dm->d);
+  }
   w.total = off;
   return w;
 }
@@ -102,12 +116,70 @@ rdl_dims clamp_w(const rdl_dims* d) {
   return c;
 }
 
+rdl_status launch_topk(const float* zeta, const float* z_all, const int32_t* q_pos, const rdl_dims* dm,
+                       int32_t* idx, float* z_sel, cudaStream_t st) {
+  const int C = dm->L / S;
+  const int warps = 4;
+  const size_t smem = (size_t)warps * C * sizeof(float);
+  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  dim3 g4((unsigned)(((long long)dm->Lq * dm->Hkv + warps - 1) / warps), dm->B);
+  count_launch();
+  topk_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
+                                            idx, z_sel);
+  return cuda_status(cudaGetLastError());
+}
+
+rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const void* w_down,
+                      const void* w_up, const float* summary, const float* entropy,
+                      const rdl_dims* dm, int32_t* idx, float* z_sel, void* workspace,
+                      cudaStream_t st) {
+  constexpr int R = 64;
+  const ScoreWs wl = score_ws(dm, RDL_BF16);
+  char* ws = static_cast<char*>(workspace);
+  float* z_all = reinterpret_cast<float*>(ws + wl.z_all);
+  float* zeta = reinterpret_cast<float*>(ws + wl.zeta);
+  __nv_bfloat16* tt = reinterpret_cast<__nv_bfloat16*>(ws + wl.tt);
+  __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(ws + wl.sb);
+  const int M = dm->B * dm->Lq, C = dm->L / S;
+  {
+    auto kern = xw_mma_kernel<R>;
+    const int smem = 2 * XW_ROWS * 128 + 2 * XW_KB * R * 2;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    count_launch();
+    kern<<<(M + XW_ROWS - 1) / XW_ROWS, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                         static_cast<const __nv_bfloat16*>(w_down), M, dm->D, tt);
+  }
+  {
+    const int smem = (R * 129 + 8 * 128) * (int)sizeof(float);
+    auto kern = sprep_kernel<R>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    count_launch();
+    kern<<<dim3((C + 31) / 32, dm->Hq, dm->B), 256, smem, st>>>(summary, static_cast<const __nv_bfloat16*>(w_up),
+                                                                 C, dm->Hq, sb);
+  }
+  {
+    auto kern = zeta_mma_kernel<R>;
+    const int smem = ZetaSmem<R>::TOTAL;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    dim3 grid((C + ZM_CH - 1) / ZM_CH, (dm->Lq + ZM_ROWS - 1) / ZM_ROWS, dm->B * dm->Hkv);
+    count_launch();
+    kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), q_pos, tt, sb, entropy, dm->Lq, dm->L,
+                                  dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
+  }
+  if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+  return launch_topk(zeta, z_all, q_pos, dm, idx, z_sel, st);
+}
+
 template <typename T>
 rdl_status score_impl(const void* q, const int32_t* q_pos, const void* x, const void* w_down,
                       const void* w_up, const float* summary, const float* entropy,
                       const rdl_dims* dm, int32_t* idx, float* z_sel, void* workspace,
                       cudaStream_t st) {
-  const ScoreWs wl = score_ws(dm);
+  const ScoreWs wl = score_ws(dm, std::is_same<T, float>::value ? RDL_F32 : RDL_BF16);
   char* ws = static_cast<char*>(workspace);
   float* t = reinterpret_cast<float*>(ws + wl.t);
   float* qres = reinterpret_cast<float*>(ws + wl.qres);
@@ -116,10 +188,15 @@ rdl_status score_impl(const void* q, const int32_t* q_pos, const void* x, const 
   const int M = dm->B * dm->Lq, N = dm->Hq * dm->d, C = dm->L / S;
   const T* qT = static_cast<const T*>(q);
   if (dm->r > 0 && x) {
-    dim3 g1((dm->r + 63) / 64, (M + 63) / 64);
     count_launch(2);
-    gemm_f32_kernel<T, T, T><<<g1, 256, 0, st>>>(static_cast<const T*>(x), static_cast<const T*>(w_down),
-                                                 (const T*)nullptr, t, M, dm->r, dm->D);
+    if (M <= 64) {
+      smallm_gemm_kernel<T, T><<<dim3((dm->r + 31) / 32, M), 256, 0, st>>>(
+          static_cast<const T*>(x), static_cast<const T*>(w_down), t, M, dm->r, dm->D);
+    } else {
+      dim3 g1((dm->r + 63) / 64, (M + 63) / 64);
+      gemm_f32_kernel<T, T, T><<<g1, 256, 0, st>>>(static_cast<const T*>(x), static_cast<const T*>(w_down),
+                                                   (const T*)nullptr, t, M, dm->r, dm->D);
+    }
     dim3 g2((N + 63) / 64, (M + 63) / 64);
     gemm_f32_kernel<float, T, T><<<g2, 256, 0, st>>>(t, static_cast<const T*>(w_up), qT, qres, M, N, dm->r);
   } else {
@@ -129,21 +206,15 @@ rdl_status score_impl(const void* q, const int32_t* q_pos, const void* x, const 
     gemm_f32_kernel<float, T, T><<<g2, 256, 0, st>>>(t, static_cast<const T*>(w_up), qT, qres, M, N, 0);
   }
   dim3 g3((C + 63) / 64, (dm->Lq + 63) / 64, dm->B * dm->Hkv);
-  count_launch(2);   // zeta + top-K
+  count_launch();    // zeta (top-K counted in launch_topk)
   if (dm->d == 128)
     zeta_kernel<128><<<g3, 256, 0, st>>>(qres, q_pos, summary, entropy, dm->Lq, dm->L, dm->Hq, dm->Hkv,
                                          dm->w, dm->lambda, z_all, zeta);
   else
     zeta_kernel<64><<<g3, 256, 0, st>>>(qres, q_pos, summary, entropy, dm->Lq, dm->L, dm->Hq, dm->Hkv,
                                         dm->w, dm->lambda, z_all, zeta);
-  const int warps = 4;
-  const size_t smem = (size_t)warps * C * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return RDL_ERR_CUDA;
-  dim3 g4((unsigned)(((long long)dm->Lq * dm->Hkv + warps - 1) / warps), dm->B);
-  topk_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
-                                            idx, z_sel);
-  return cuda_status(cudaGetLastError());
+  if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+  return launch_topk(zeta, z_all, q_pos, dm, idx, z_sel, st);
 }
 
 template <typename T, bool ROUTE>
@@ -206,7 +277,7 @@ const char* rdl_status_string(rdl_status s) {
 
 size_t rdl_workspace_bytes(int which, const rdl_dims* dims, rdl_dtype dtype) {
   if (!route_dims_ok(dims) || !dtype_ok(dtype)) return 0;
-  if (which == RDL_WS_SCORE) return score_ws(dims).total;
+  if (which == RDL_WS_SCORE) return score_ws(dims, dtype).total;
   if (which == RDL_WS_ATTN) return attn_ws(dims, dtype).total;
   return 0;
 }
@@ -254,10 +325,12 @@ rdl_status rdl_route_score_topk(const void* q, const int32_t* q_pos, const void*
       (residual && (!aligned16(x) || !aligned16(w_down) || !aligned16(w_up))) ||
       (q_pos && !aligned16(q_pos)))
     return RDL_ERR_INVALID_ARG;
-  if (ws_bytes < score_ws(dims).total) return RDL_ERR_WORKSPACE;
   rdl_dims dm = clamp_w(dims);
   if (!residual) dm.r = 0;
+  if (ws_bytes < score_ws(&dm, dtype).total) return RDL_ERR_WORKSPACE;
   const cudaStream_t st = as_stream(stream);
+  if (fast_score(&dm, dtype))
+    return score_fast(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel, workspace, st);
   return dtype == RDL_BF16 ? score_impl<__nv_bfloat16>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx,
                                                        z_sel, workspace, st)
                            : score_impl<float>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel,

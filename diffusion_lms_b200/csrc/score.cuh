@@ -70,6 +70,34 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const TA* __restrict__ A,
   }
 }
 
+// Out[M,N] = A[M,Kd] * B[Kd,N] for few rows (decode blocks): one CTA per (row, 32 columns),
+// the K loop split over 256 threads and reduced in shared memory.
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) smallm_gemm_kernel(const TA* __restrict__ A,
+                                                          const TB* __restrict__ Bm,
+                                                          float* __restrict__ Out, int M, int N,
+                                                          int Kd) {
+  __shared__ float red[256][33];
+  const int m = blockIdx.y, n0 = blockIdx.x * 32, tid = threadIdx.x;
+  float acc[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+  for (int k = tid; k < Kd; k += 256) {
+    const float a = IO<TA>::ld(A + (size_t)m * Kd + k);
+    const TB* br = Bm + (size_t)k * N + n0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = fmaf(a, (n0 + j < N) ? IO<TB>::ld(br + j) : 0.f, acc[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) red[tid][j] = acc[j];
+  __syncthreads();
+  if (tid < 32) {
+    float sum = 0.f;
+    for (int t = 0; t < 256; ++t) sum += red[t][tid];
+    if (n0 + tid < N) Out[(size_t)m * N + n0 + tid] = sum;
+  }
+}
+
 // --------------------------------------------------------------------------- stage 2
 // One CTA per (chunk tile of 64, query tile of 64, b*Hkv + g).
 template <int D>
