@@ -206,6 +206,71 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
+    """128K decode block: rdl_route_score_topk + rdl_route_attn with cached summaries,
+    captured once in a CUDA graph and replayed; L2 flushed between replays (untimed)."""
+    import torch
+    from diffusion_lms_b200 import api, rdl
+    from diffusion_lms_b200 import workloads as W
+    wd = W.decode_128k(seed=rank_seed(3, rank))
+    dinp = api.to_device(wd, dev)
+    dout = api.alloc_outputs(dinp.dims, dinp.dtype, dev)
+    api.summary_pool(dinp, dout, stream=stream)
+
+    def dstep():
+        api.score_topk(dinp, dout, stream=stream)
+        api.route_attn(dinp, dout, stream=stream)
+
+    for _ in range(args.warmup):
+        dstep()
+    torch.cuda.synchronize()
+    # per-call split (eager launches)
+    eag = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for s_ in range(args.steps):
+        flush.zero_()
+        e = eag[s_]
+        e[0].record(stream)
+        api.score_topk(dinp, dout, stream=stream)
+        e[1].record(stream)
+        api.route_attn(dinp, dout, stream=stream)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    dper = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in eag])
+    # graph replay of the whole step
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            api.score_topk(dinp, dout, stream=cs)
+            api.route_attn(dinp, dout, stream=cs)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s_ in range(args.steps):
+        flush.zero_()
+        gev[s_][0].record(stream)
+        g.replay()
+        gev[s_][1].record(stream)
+    torch.cuda.synchronize()
+    gms = np.array([e[0].elapsed_time(e[1]) for e in gev])
+    d_ms = max_over_ranks(float(np.median(gms)), world, dev) if world > 1 else float(np.median(gms))
+    assert rdl.rdl_last_device_status() == rdl.OK
+    db = decode_bytes(dinp.dims, dout.idx.cpu().numpy())
+    d_ach = db["total"] / (d_ms / 1e3) / 1e9
+    del g
+    return {"workload": wd.name, "ms_per_step": d_ms, "timing": "CUDA-graph replay, median",
+            "eager_ms_per_step": float(np.median(dper.sum(axis=1))),
+            "score_ms": float(np.median(dper[:, 0])), "attn_ms": float(np.median(dper[:, 1])),
+            "query_tokens_per_s": world * 32 / (d_ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": d_ach / pk["hbm_gbs"], "algorithmic_bytes": db["total"],
+                         "unique_group_chunk_pairs": db["unique_pairs"],
+                         "peak_source": f"hbm_gbs ({pk_kind})"}}
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def main():
@@ -217,6 +282,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=96)
     ap.add_argument("--cpu-rows", type=int, default=96)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the 128K decode block (profiling aid)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -250,6 +317,13 @@ def main():
 
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    pk, pk_kind = peaks()
+    if args.decode_only:
+        dec = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"decode_128k": dec}), flush=True)
+        return
 
     # ---------------- 16K prefill route layer (the headline workload)
     wl = W.prefill_16k(seed=rank_seed(2, rank))
@@ -297,7 +371,6 @@ def main():
     idx_np = out.idx.cpu().numpy()
     fl_attn = attn_flops(wl.dims, None, idx_np)
     fl_score = score_flops(wl.dims)
-    pk, pk_kind = peaks()
     calls = {"rdl_summary_pool": float(call_ms[0]), "rdl_route_score_topk": float(call_ms[1]),
              "rdl_route_attn": float(call_ms[2])}
     dominant = max(calls, key=calls.get)
@@ -355,41 +428,7 @@ def main():
     if not args.no_decode:
         del inp, out
         torch.cuda.empty_cache()
-        wd = W.decode_128k(seed=rank_seed(3, rank))
-        dinp = api.to_device(wd, dev)
-        dout = api.alloc_outputs(dinp.dims, dinp.dtype, dev)
-        api.summary_pool(dinp, dout, stream=stream)
-
-        def dstep():
-            api.score_topk(dinp, dout, stream=stream)
-            api.route_attn(dinp, dout, stream=stream)
-
-        for _ in range(args.warmup):
-            dstep()
-        torch.cuda.synchronize()
-        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        barrier()
-        for s_ in range(args.steps):
-            flush.zero_()
-            e = dev_ev[s_]
-            e[0].record(stream)
-            api.score_topk(dinp, dout, stream=stream)
-            e[1].record(stream)
-            api.route_attn(dinp, dout, stream=stream)
-            e[2].record(stream)
-        torch.cuda.synchronize()
-        dper = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in dev_ev])
-        d_ms = max_ranks(float(np.median(dper.sum(axis=1))))
-        db = decode_bytes(dinp.dims, dout.idx.cpu().numpy())
-        d_ach = db["total"] / (d_ms / 1e3) / 1e9
-        decode = {"workload": wd.name, "ms_per_step": d_ms,
-                  "score_ms": float(np.median(dper[:, 0])), "attn_ms": float(np.median(dper[:, 1])),
-                  "query_tokens_per_s": world * 32 / (d_ms / 1e3),
-                  "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                               "frac": d_ach / pk["hbm_gbs"], "algorithmic_bytes": db["total"],
-                               "unique_group_chunk_pairs": db["unique_pairs"],
-                               "peak_source": f"hbm_gbs ({pk_kind})"}}
-        assert rdl.rdl_last_device_status() == rdl.OK
+        decode = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
 
     # ---------------- CPU baseline (rank 0, oracle on a bounded sample)
     cpu = None

@@ -84,6 +84,7 @@ class Outputs:
     lse: torch.Tensor
     ws_score: torch.Tensor
     ws_attn: torch.Tensor
+    ws_swa: torch.Tensor
     extra: dict = field(default_factory=dict)
 
 
@@ -92,6 +93,7 @@ def alloc_outputs(dims: rdl.Dims, dtype: str, device="cuda") -> Outputs:
     dev = torch.device(device)
     ws_s = rdl.workspace_bytes(rdl.WS_SCORE, dims, dtype)
     ws_a = rdl.workspace_bytes(rdl.WS_ATTN, dims, dtype)
+    ws_w = rdl.workspace_bytes(rdl.WS_SWA, dims, dtype)
     return Outputs(
         s=torch.empty(dims.B, dims.Hq, C, dims.d, dtype=torch.float32, device=dev),
         H=torch.empty(dims.B, dims.Hq, C, dtype=torch.float32, device=dev),
@@ -101,6 +103,7 @@ def alloc_outputs(dims: rdl.Dims, dtype: str, device="cuda") -> Outputs:
         lse=torch.full((dims.B, dims.Hq, dims.Lq), float("nan"), dtype=torch.float32, device=dev),
         ws_score=torch.empty(max(ws_s, 256), dtype=torch.uint8, device=dev),
         ws_attn=torch.empty(max(ws_a, 256), dtype=torch.uint8, device=dev),
+        ws_swa=torch.empty(max(ws_w, 256), dtype=torch.uint8, device=dev),
     )
 
 
@@ -125,7 +128,7 @@ def route_attn(inp: DeviceInputs, out: Outputs, stream=None):
 
 def swa_attn(inp: DeviceInputs, out: Outputs, stream=None):
     rdl.rdl_swa_attn(inp.q, inp.q_pos, inp.k, inp.v, inp.dims, inp.dtype, out.o, out.lse,
-                     stream=stream)
+                     out.ws_swa, stream=stream)
 
 
 def route_layer(inp: DeviceInputs, out: Outputs, *, with_summary=True, stream=None):

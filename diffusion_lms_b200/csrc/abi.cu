@@ -11,8 +11,11 @@
 #include "summary_pool.cuh"
 #include "score.cuh"
 #include "score_mma.cuh"
+#include "decode_score.cuh"
 #include "window_attn.cuh"
 #include "chunk_attn.cuh"
+#include "tmap.cuh"
+#include "chunk_tc.cuh"
 
 using namespace rdl;
 
@@ -55,11 +58,23 @@ bool route_dims_ok(const rdl_dims* dm) {
 bool fast_attn(const rdl_dims* dm, rdl_dtype t) {
   return t == RDL_BF16 && dm->d == 128 && dm->Hq / dm->Hkv <= 8;
 }
+// Chunk splits of the selected-chunk pass when there are few (row, group) items.
 int attn_splits(const rdl_dims* dm) {
   const long long items = (long long)dm->B * dm->Lq * dm->Hkv;
   if (items >= 4096) return 1;
   int ns = (int)((4096 + items - 1) / items);
-  return ns < 8 ? (ns < dm->K ? ns : dm->K) : (8 < dm->K ? 8 : dm->K);
+  if (ns > 16) ns = 16;
+  return ns < dm->K ? ns : dm->K;
+}
+// Key splits of the window pass when there are few 16-row tiles (decode blocks).
+int window_splits(const rdl_dims* dm) {
+  if (dm->w < 0) return 1;
+  const long long ctas = (long long)dm->B * ((dm->Lq + WIN_ROWS - 1) / WIN_ROWS) * dm->Hkv;
+  if (ctas >= 148) return 1;
+  const long long want = (296 + ctas - 1) / ctas;
+  const long long blocks = (2LL * dm->w + WIN_ROWS + WIN_KEYS - 1) / WIN_KEYS + 1;
+  long long ns = want < blocks ? want : blocks;
+  return ns < 1 ? 1 : (int)ns;
 }
 
 // The tensor-core score path: bf16, d = 128, rank 64 residual with D % 64 == 0, and
@@ -69,8 +84,10 @@ bool fast_score(const rdl_dims* dm, rdl_dtype t) {
   return t == RDL_BF16 && dm->d == 128 && dm->r == 64 && dm->D % 64 == 0 && dm->Hq / dm->Hkv <= 8 &&
          dm->Lq >= kFastScoreMinRows;
 }
+// decode blocks: few rows, head dim 128 -> the decode score path
+bool decode_score_path(const rdl_dims* dm) { return dm->d == 128 && dm->Lq <= 64; }
 struct ScoreWs {
-  size_t t, qres, z_all, zeta, tt, sb, total;
+  size_t t, qres, z_all, zeta, tt, sb, tpart, total;
 };
 ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   const size_t C = dm->L / S;
@@ -84,6 +101,10 @@ ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   } else {
     w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
     w.qres = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * dm->Hq * dm->d);
+    if (decode_score_path(dm) && dm->r > 0) {
+      const size_t nsl = (dm->D + DQ_KS - 1) / DQ_KS;
+      w.tpart = off; off += align256(sizeof(float) * nsl * dm->B * dm->Lq * dm->r);
+    }
   }
   w.total = off;
   return w;
@@ -96,13 +117,23 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
   if (!fast_attn(dm, t)) return w;
   const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
   size_t off = 0;
-  w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d);
-  w.lam_loc = off; off += align256(sizeof(float) * rows);
+  const int nsw = window_splits(dm);
+  w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d * nsw);
+  w.lam_loc = off; off += align256(sizeof(float) * rows * nsw);
   w.o_acc = off;
   const int ns = attn_splits(dm);
   if (ns > 1) off += align256(sizeof(float) * rows * dm->d * ns);
   w.total = off;
   return w;
+}
+
+// Sliding-window workspace: key-split partials when the row count is small (else none).
+size_t swa_ws(const rdl_dims* dm, rdl_dtype t) {
+  if (!fast_attn(dm, t) || dm->w < 0) return 0;
+  const int nsw = window_splits(dm);
+  if (nsw <= 1) return 0;
+  const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
+  return align256(sizeof(float) * rows * dm->d * nsw) + align256(sizeof(float) * rows * nsw);
 }
 
 rdl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RDL_OK : RDL_ERR_CUDA; }
@@ -119,14 +150,26 @@ rdl_dims clamp_w(const rdl_dims* d) {
 rdl_status launch_topk(const float* zeta, const float* z_all, const int32_t* q_pos, const rdl_dims* dm,
                        int32_t* idx, float* z_sel, cudaStream_t st) {
   const int C = dm->L / S;
+  if ((long long)dm->B * dm->Lq * dm->Hkv <= 1024) {
+    // few rows: a CTA per (row, group)
+    const size_t smem = (size_t)C * sizeof(uint32_t);
+    if (cudaFuncSetAttribute(topk_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return RDL_ERR_CUDA;
+    count_launch();
+    topk_cta_kernel<<<dim3(dm->Lq * dm->Hkv, dm->B), 256, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq,
+                                                                      dm->Hkv, dm->K, idx, z_sel);
+    return cuda_status(cudaGetLastError());
+  }
   const int warps = 4;
-  const size_t smem = (size_t)warps * C * sizeof(float);
-  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  const size_t smem = (size_t)warps * (C + 256) * sizeof(uint32_t);
+  if (cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return RDL_ERR_CUDA;
   dim3 g4((unsigned)(((long long)dm->Lq * dm->Hkv + warps - 1) / warps), dm->B);
   count_launch();
-  topk_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
-                                            idx, z_sel);
+  topk_radix_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
+                                                  idx, z_sel);
   return cuda_status(cudaGetLastError());
 }
 
@@ -187,6 +230,35 @@ rdl_status score_impl(const void* q, const int32_t* q_pos, const void* x, const 
   float* zeta = reinterpret_cast<float*>(ws + wl.zeta);
   const int M = dm->B * dm->Lq, N = dm->Hq * dm->d, C = dm->L / S;
   const T* qT = static_cast<const T*>(q);
+  if (decode_score_path(dm)) {
+    // decode blocks: fused residual query per row, then a tensor-core pass that streams
+    // the cached summaries once
+    const bool res = dm->r > 0 && x;
+    if (cudaFuncSetAttribute(dec_tpart_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_TPART_SMEM) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(dec_qres_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_QRES_SMEM) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(decode_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DS_SMEM) !=
+            cudaSuccess)
+      return RDL_ERR_CUDA;
+    const int rowblocks = (M + DQ_ROWS - 1) / DQ_ROWS;
+    if (res) {
+      // t = x W_down by 64-wide slices of D, then summed
+      float* tpart = reinterpret_cast<float*>(ws + wl.tpart);
+      const int nsl = (dm->D + DQ_KS - 1) / DQ_KS;
+      count_launch(2);
+      dec_tpart_kernel<T><<<dim3(nsl, rowblocks), 256, DQ_TPART_SMEM, st>>>(
+          static_cast<const T*>(x), static_cast<const T*>(w_down), M, dm->D, dm->r, tpart);
+      dec_tsum_kernel<<<(M * dm->r + 255) / 256, 256, 0, st>>>(tpart, nsl, M * dm->r, t);
+    }
+    count_launch(2);
+    dec_qres_kernel<T><<<dim3((N + 127) / 128, rowblocks), 256, DQ_QRES_SMEM, st>>>(
+        qT, res ? t : nullptr, static_cast<const T*>(w_up), M, res ? dm->r : 0, N, qres);
+    decode_score_kernel<<<dim3((C + DS_CH - 1) / DS_CH, dm->B * dm->Hkv), 128, DS_SMEM, st>>>(
+        qres, q_pos, summary, entropy, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
+    if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+    return launch_topk(zeta, z_all, q_pos, dm, idx, z_sel, st);
+  }
   if (dm->r > 0 && x) {
     count_launch(2);
     if (M <= 64) {
@@ -238,18 +310,18 @@ rdl_status generic_attn(const void* q, const int32_t* q_pos, const void* k, cons
 template <int MODE>
 rdl_status launch_window_mma(const void* q, const int32_t* q_pos, const void* k, const void* v,
                              const rdl_dims* dm, void* o, float* lse, float* o_loc, float* lam_loc,
-                             cudaStream_t st) {
+                             int nsplit, cudaStream_t st) {
   const int G = dm->Hq / dm->Hkv;
   const size_t smem = window_mma_smem(G);
   auto kern = window_mma_kernel<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return RDL_ERR_CUDA;
-  dim3 grid((dm->Lq + WIN_ROWS - 1) / WIN_ROWS, dm->B * dm->Hkv);
+  dim3 grid((dm->Lq + WIN_ROWS - 1) / WIN_ROWS, dm->B * dm->Hkv, nsplit);
   count_launch();
   kern<<<grid, 32 * G, smem, st>>>(static_cast<const __nv_bfloat16*>(q), q_pos,
                                    static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
                                    dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->w, static_cast<__nv_bfloat16*>(o), lse,
-                                   o_loc, lam_loc);
+                                   o_loc, lam_loc, nsplit);
   return cuda_status(cudaGetLastError());
 }
 
@@ -279,6 +351,7 @@ size_t rdl_workspace_bytes(int which, const rdl_dims* dims, rdl_dtype dtype) {
   if (!route_dims_ok(dims) || !dtype_ok(dtype)) return 0;
   if (which == RDL_WS_SCORE) return score_ws(dims, dtype).total;
   if (which == RDL_WS_ATTN) return attn_ws(dims, dtype).total;
+  if (which == RDL_WS_SWA) return swa_ws(dims, dtype);
   return 0;
 }
 
@@ -361,10 +434,31 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
   float* o_loc = reinterpret_cast<float*>(ws + wl.o_loc);
   float* lam_loc = reinterpret_cast<float*>(ws + wl.lam_loc);
   float* o_acc = reinterpret_cast<float*>(ws + wl.o_acc);
-  rdl_status s = launch_window_mma<1>(q, q_pos, k, v, dims, nullptr, nullptr, o_loc, lam_loc, st);
+  const int nsw = window_splits(dims);
+  rdl_status s = launch_window_mma<1>(q, q_pos, k, v, dims, nullptr, nullptr, o_loc, lam_loc, nsw, st);
   if (s != RDL_OK) return s;
   const int ns = attn_splits(dims);
   const size_t rows = (size_t)dims->B * dims->Lq * dims->Hq;
+  const int C = dims->L / S;
+  if (ns == 1 && C <= CT_MAXC && dims->K <= CT_MAXK) {
+    // prefill: tcgen05 kernel, 48-row tiles sharing each selected chunk's K/V
+    CUtensorMap mq, mk, mv;
+    const unsigned long long qrows = (unsigned long long)dims->B * dims->Lq * dims->Hq;
+    const unsigned long long kvrows = (unsigned long long)dims->B * dims->Hkv * dims->L;
+    if (make_tmap_bf16(&mq, q, qrows, 128, 64, 8) && make_tmap_bf16(&mk, k, kvrows, 128, 64, 64) &&
+        make_tmap_bf16(&mv, v, kvrows, 128, 64, 64)) {
+      if (cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CT_SMEM) !=
+          cudaSuccess)
+        return RDL_ERR_CUDA;
+      dim3 grid((dims->Lq + CT_TQ - 1) / CT_TQ, dims->B * dims->Hkv);
+      count_launch();
+      chunk_tc_kernel<<<grid, CT_THREADS, CT_SMEM, st>>>(mq, mk, mv, q_pos, idx, z_sel, o_loc, lam_loc, nsw,
+                                                         dims->L, dims->Lq, dims->Hq, dims->Hkv, dims->K,
+                                                         dims->w, dims->flags, static_cast<__nv_bfloat16*>(o),
+                                                         lse);
+      return cuda_status(cudaGetLastError());
+    }
+  }
   const size_t smem = (size_t)CH_WARPS * CH_WARP_SMEM;
   if (cudaFuncSetAttribute(chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -375,7 +469,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
   chunk_mma_kernel<<<grid, CH_WARPS * 32, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), q_pos, static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), idx, z_sel, o_loc, lam_loc, dims->L, dims->Lq, dims->Hq, dims->Hkv,
-      dims->K, dims->w, ns, dims->flags, static_cast<__nv_bfloat16*>(o), lse, o_acc);
+      dims->K, dims->w, ns, dims->flags, static_cast<__nv_bfloat16*>(o), lse, o_acc, nsw);
   if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
   if (ns > 1) {
     const long long n = (long long)rows * dims->d;
@@ -388,7 +482,8 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
 }
 
 rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, const void* v,
-                        const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse, void* stream) {
+                        const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse, void* workspace,
+                        size_t ws_bytes, void* stream) {
   if (!dims_ok(dims) || !dtype_ok(dtype) || dims->w < 0) return RDL_ERR_INVALID_ARG;
   if (!q_pos && dims->Lq != dims->L) return RDL_ERR_INVALID_ARG;
   if (!q || !k || !v || !o) return RDL_ERR_INVALID_ARG;
@@ -402,7 +497,23 @@ rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, cons
     return dtype == RDL_BF16 ? generic_attn<__nv_bfloat16, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st)
                              : generic_attn<float, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st);
   }
-  return launch_window_mma<0>(q, q_pos, k, v, dims, o, lse, nullptr, nullptr, st);
+  const size_t need = swa_ws(dims, dtype);
+  if (need == 0 || !workspace) return launch_window_mma<0>(q, q_pos, k, v, dims, o, lse, nullptr, nullptr, 1, st);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RDL_ERR_INVALID_ARG;
+  if (ws_bytes < need) return RDL_ERR_WORKSPACE;
+  // few rows: key-split partials, then the combine pass
+  const int nsw = window_splits(dims);
+  const size_t rows = (size_t)dims->B * dims->Lq * dims->Hq;
+  float* o_part = static_cast<float*>(workspace);
+  float* l_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(sizeof(float) * rows * dims->d * nsw));
+  rdl_status s = launch_window_mma<0>(q, q_pos, k, v, dims, nullptr, nullptr, o_part, l_part, nsw, st);
+  if (s != RDL_OK) return s;
+  const long long n = (long long)rows * dims->d;
+  const int blocks = (int)((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048);
+  count_launch();
+  window_combine_kernel<<<blocks, 256, 0, st>>>(o_part, l_part, nsw, dims->B, dims->Lq, dims->Hq,
+                                                static_cast<__nv_bfloat16*>(o), lse);
+  return cuda_status(cudaGetLastError());
 }
 
 rdl_status rdl_last_device_status(void* stream) {

@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(CH_WARPS * 32) chunk_mma_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ z_sel,
     const float* __restrict__ o_loc, const float* __restrict__ lam_loc, int L, int Lq, int Hq,
     int Hkv, int K, int w, int nsplit, int flags, __nv_bfloat16* __restrict__ o,
-    float* __restrict__ lse, float* __restrict__ o_acc) {
+    float* __restrict__ lse, float* __restrict__ o_acc, int nsw) {
   constexpr int D = 128;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -71,21 +71,82 @@ __global__ void __launch_bounds__(CH_WARPS * 32) chunk_mma_kernel(
   const int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
   const size_t zA = ((size_t)(b * Hq + g * G + (vA ? hA : 0)) * Lq + i) * K;
   const size_t zB = ((size_t)(b * Hq + g * G + (vB ? hB : 0)) * Lq + i) * K;
-  const float lamA = vA ? lam_loc[(size_t)(b * Hq + g * G + hA) * Lq + i] : 0.f;
-  const float lamB = vB ? lam_loc[(size_t)(b * Hq + g * G + hB) * Lq + i] : 0.f;
+  // window log-sum-exp: merge the key-split planes, lambda = LSE_s lambda_s
+  const size_t plane_l = (size_t)gridDim.y * Hq * Lq;
+  const size_t liA = (size_t)(b * Hq + g * G + (vA ? hA : 0)) * Lq + i;
+  const size_t liB = (size_t)(b * Hq + g * G + (vB ? hB : 0)) * Lq + i;
+  float lamA = -INFINITY, lamB = -INFINITY;
+  {
+    // lanes sharing tq split the window planes (nsw <= 8 * lanes-per-head)
+    float la = -INFINITY, lb = -INFINITY, mA = -INFINITY, mB = -INFINITY;
+    float lva[2], lvb[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int sw = gq + 8 * u;
+      lva[u] = sw < nsw ? lam_loc[sw * plane_l + liA] : -INFINITY;
+      lvb[u] = sw < nsw ? lam_loc[sw * plane_l + liB] : -INFINITY;
+      mA = fmaxf(mA, lva[u]);
+      mB = fmaxf(mB, lvb[u]);
+    }
+    for (int sw = gq + 16; sw < nsw; sw += 8) {
+      mA = fmaxf(mA, lam_loc[sw * plane_l + liA]);
+      mB = fmaxf(mB, lam_loc[sw * plane_l + liB]);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, off));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, off));
+    }
+    float sA = 0.f, sB = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (lva[u] != -INFINITY) sA += expf(lva[u] - mA);
+      if (lvb[u] != -INFINITY) sB += expf(lvb[u] - mB);
+    }
+    for (int sw = gq + 16; sw < nsw; sw += 8) {
+      const float a = lam_loc[sw * plane_l + liA], bb = lam_loc[sw * plane_l + liB];
+      if (a != -INFINITY) sA += expf(a - mA);
+      if (bb != -INFINITY) sB += expf(bb - mB);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      sA += __shfl_xor_sync(0xffffffffu, sA, off);
+      sB += __shfl_xor_sync(0xffffffffu, sB, off);
+    }
+    (void)la; (void)lb;
+    if (vA && sA > 0.f) lamA = mA + logf(sA);
+    if (vB && sB > 0.f) lamB = mB + logf(sB);
+  }
+  // the 8 lanes sharing tq (same heads) split the K slots: loads in flight together
+  float zvA[8], zvB[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int kk = gq + 8 * u;
+    zvA[u] = kk < K ? z_sel[zA + kk] : -INFINITY;
+    zvB[u] = kk < K ? z_sel[zB + kk] : -INFINITY;
+  }
   float MA = lamA, MB = lamB;
-  for (int kk = 0; kk < K; ++kk) {
-    MA = fmaxf(MA, z_sel[zA + kk]);
-    MB = fmaxf(MB, z_sel[zB + kk]);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) { MA = fmaxf(MA, zvA[u]); MB = fmaxf(MB, zvB[u]); }
+  for (int kk = gq + 64; kk < K; kk += 8) { MA = fmaxf(MA, z_sel[zA + kk]); MB = fmaxf(MB, z_sel[zB + kk]); }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    MA = fmaxf(MA, __shfl_xor_sync(0xffffffffu, MA, off));
+    MB = fmaxf(MB, __shfl_xor_sync(0xffffffffu, MB, off));
   }
   if (MA == -INFINITY) MA = 0.f;   // no part at all (cannot happen for valid selections)
   if (MB == -INFINITY) MB = 0.f;
-  float ZA = (lamA == -INFINITY) ? 0.f : expf(lamA - MA);
-  float ZB = (lamB == -INFINITY) ? 0.f : expf(lamB - MB);
-  for (int kk = 0; kk < K; ++kk) {
-    ZA += expf(z_sel[zA + kk] - MA);
-    ZB += expf(z_sel[zB + kk] - MB);
+  float ZA = 0.f, ZB = 0.f;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) { ZA += expf(zvA[u] - MA); ZB += expf(zvB[u] - MB); }
+  for (int kk = gq + 64; kk < K; kk += 8) { ZA += expf(z_sel[zA + kk] - MA); ZB += expf(z_sel[zB + kk] - MB); }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    ZA += __shfl_xor_sync(0xffffffffu, ZA, off);
+    ZB += __shfl_xor_sync(0xffffffffu, ZB, off);
   }
+  ZA += (lamA == -INFINITY) ? 0.f : expf(lamA - MA);
+  ZB += (lamB == -INFINITY) ? 0.f : expf(lamB - MB);
   const float invZA = ZA > 0.f ? 1.f / ZA : 0.f, invZB = ZB > 0.f ? 1.f / ZB : 0.f;
 
   const int per = (K + nsplit - 1) / nsplit;
@@ -227,17 +288,23 @@ __global__ void __launch_bounds__(CH_WARPS * 32) chunk_mma_kernel(
 
   // ---- local window part (one split adds it)
   if (split == 0) {
-    const float wA = (vA && lamA != -INFINITY) ? expf(lamA - MA) * invZA : 0.f;
-    const float wB = (vB && lamB != -INFINITY) ? expf(lamB - MB) * invZB : 0.f;
-    const float* olA = o_loc + ((size_t)(b * Lq + i) * Hq + g * G + (vA ? hA : 0)) * D;
-    const float* olB = o_loc + ((size_t)(b * Lq + i) * Hq + g * G + (vB ? hB : 0)) * D;
+    // each key-split plane of the window enters with mass e^{lambda_s - M}/Zs
+    const size_t plane = (size_t)gridDim.y * Lq * Hq * D;
+    for (int sw = 0; sw < nsw; ++sw) {
+      const float lsA = vA ? lam_loc[sw * plane_l + liA] : -INFINITY;
+      const float lsB = vB ? lam_loc[sw * plane_l + liB] : -INFINITY;
+      const float wA = (lsA != -INFINITY) ? expf(lsA - MA) * invZA : 0.f;
+      const float wB = (lsB != -INFINITY) ? expf(lsB - MB) * invZB : 0.f;
+      const float* olA = o_loc + sw * plane + ((size_t)(b * Lq + i) * Hq + g * G + (vA ? hA : 0)) * D;
+      const float* olB = o_loc + sw * plane + ((size_t)(b * Lq + i) * Hq + g * G + (vB ? hB : 0)) * D;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
+      for (int mt = 0; mt < 8; ++mt) {
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int dd = mt * 16 + gq + 8 * hr;
-        if (vA) oacc[mt][2 * hr] += wA * olA[dd];
-        if (vB) oacc[mt][2 * hr + 1] += wB * olB[dd];
+        for (int hr = 0; hr < 2; ++hr) {
+          const int dd = mt * 16 + gq + 8 * hr;
+          if (wA != 0.f) oacc[mt][2 * hr] += wA * olA[dd];
+          if (wB != 0.f) oacc[mt][2 * hr + 1] += wB * olB[dd];
+        }
       }
     }
     if (lse && gq == 0) {

@@ -1,0 +1,471 @@
+// Selected-chunk attention of the route layer on tcgen05 tensor cores (prefill).
+//
+// Same partition as chunk_mma_kernel ([v2] Figure 3 caption: the selected chunk scores and
+// the window's log-sum-exp share one softmax partition; a second softmax spreads each
+// chunk's mass over its 63 content tokens), organised so that one load of a chunk's K/V
+// serves every query of a 48-row tile that selected it:
+//
+//   CTA = (48 consecutive query rows, one KV group).  The tile's (row, slot) selections are
+//   bucketed by chunk (counting sort in shared memory).  For every chunk in the union, in
+//   ascending order, the K/V slab (2 x 16 KB) arrives by TMA, and the rows that selected it
+//   are processed 8 queries (64 rows = 8 x 8 padded heads) at a time:
+//     S   = Q_rows K_c^T        tcgen05.mma M=64 N=64 K=128 -> TMEM (double-buffered)
+//     P   = e^{S - max} * w_{i,h,c} / l   over the 63 content keys, written to smem (bf16)
+//     O^T[:, 8q..8q+8) += V_c^T P_q^T    tcgen05.mma M=128 (head dim) N=8 K=64, one per
+//                                         query, accumulating straight into that query's
+//                                         home columns of TMEM (no scatter pass)
+//   where w = e^{z_{i,h,c} - M}/Z is fixed up front (z_sel and the window lse are inputs).
+//   The home accumulators O^T [128 lanes x 48*8 columns] stay in TMEM for the whole tile;
+//   the epilogue adds the window part and writes o once.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (one thread) and
+// TMEM owner, warps 2-5 = softmax + epilogue (one per TMEM lane quarter).
+// Every wait is bounded; on a timeout the kernel records RDL_ERR_TIMEOUT, every role
+// stops, TMEM is freed and the kernel returns.
+#pragma once
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace rdl {
+
+constexpr int CT_TQ = 48;                  // query rows per CTA
+constexpr int CT_HP = 8;                   // rows per query in S / columns per query in TMEM
+constexpr int CT_QP = 8;                   // queries per MMA pass (M = 64)
+constexpr int CT_NSLOT = 3;                // K/V ring depth
+constexpr int CT_MAXC = 2048;              // chunks (L <= 131072)
+constexpr int CT_MAXK = 64;
+constexpr int CT_HOME = CT_TQ * CT_HP;     // 384 home columns
+constexpr int CT_SCOL = CT_HOME;           // S buffers at 384 and 448
+constexpr int CT_THREADS = 192;
+
+// shared-memory map (bytes from the 1024-aligned base)
+constexpr int CT_OFF_KV = 0;                                   // slot s: K at s*32K, V at +16K
+constexpr int CT_OFF_A = CT_OFF_KV + CT_NSLOT * 32768;         // 2 x 16 KB gathered Q rows
+constexpr int CT_OFF_P = CT_OFF_A + 2 * 16384;                 // 2 x 8 KB P tiles
+constexpr int CT_OFF_BAR = CT_OFF_P + 2 * 8192;                // mbarriers
+constexpr int CT_NBAR = 2 * CT_NSLOT + 2 * 5 + 1;
+constexpr int CT_OFF_MISC = CT_OFF_BAR + 256;                  // tmem base, abort, nunion
+constexpr int CT_OFF_CNT = CT_OFF_MISC + 128;                  // counts / cursor [MAXC] int
+constexpr int CT_OFF_OFS = CT_OFF_CNT + CT_MAXC * 4;           // offsets [MAXC] int
+constexpr int CT_OFF_UNI = CT_OFF_OFS + CT_MAXC * 4;           // union [MAXC] u32
+constexpr int CT_OFF_ENT = CT_OFF_UNI + CT_MAXC * 4;           // entries [TQ*MAXK] u16
+constexpr int CT_OFF_MW = CT_OFF_ENT + CT_TQ * CT_MAXK * 2;    // M [TQ][8]
+constexpr int CT_OFF_IZ = CT_OFF_MW + CT_TQ * 8 * 4;           // 1/Z [TQ][8]
+constexpr int CT_OFF_WW = CT_OFF_IZ + CT_TQ * 8 * 4;           // window mass [TQ][8]
+constexpr int CT_OFF_POS = CT_OFF_WW + CT_TQ * 8 * 4;          // positions [TQ]
+constexpr int CT_OFF_PART = CT_OFF_POS + CT_TQ * 4;            // scan partials [192][2]
+constexpr int CT_SMEM = CT_OFF_PART + CT_THREADS * 8 + 1024;   // + alignment slack
+
+struct CtBars {
+  uint64_t* full;    // [NSLOT] K/V landed
+  uint64_t* empty;   // [NSLOT] K/V slot released (MMA commit)
+  uint64_t* afull;   // [2] gathered Q rows landed
+  uint64_t* aempty;  // [2] Q tile consumed by MMA1 (commit)
+  uint64_t* sfull;   // [2] S ready (commit)
+  uint64_t* sempty;  // [2] S read by the softmax warps (4 arrivals)
+  uint64_t* pfull;   // [2] P written (4 arrivals)
+  uint64_t* pempty;  // [2] P consumed by the PV MMAs (commit)
+  uint64_t* done;    // all MMAs complete (commit)
+};
+
+// bounded wait that also gives up as soon as another role has aborted
+__device__ __forceinline__ bool ct_wait(uint64_t* bar, unsigned parity, volatile int* abort_flag) {
+  for (unsigned it = 0; it < tc::kSpinLimit; ++it) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && *abort_flag) return false;
+  }
+  record_status(RDL_ERR_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ uint32_t ct_union(int c, int start, int cnt) {
+  return (uint32_t)c | ((uint32_t)start << 12) | ((uint32_t)cnt << 24);
+}
+
+__global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
+    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+    const __grid_constant__ CUtensorMap map_v, const int32_t* __restrict__ q_pos,
+    const int32_t* __restrict__ idx, const float* __restrict__ z_sel, const float* __restrict__ o_loc,
+    const float* __restrict__ lam_loc, int nsw, int L, int Lq, int Hq, int Hkv, int K, int w, int flags,
+    __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  extern __shared__ unsigned char ct_raw[];
+  unsigned char* sm = ct_raw + ((1024u - (smem_u32(ct_raw) & 1023u)) & 1023u);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = Hq / Hkv, C = L / S;
+  const int i0 = blockIdx.x * CT_TQ;
+  const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CT_OFF_BAR);
+  CtBars B{bars, bars + CT_NSLOT, bars + 2 * CT_NSLOT, bars + 2 * CT_NSLOT + 2, bars + 2 * CT_NSLOT + 4,
+           bars + 2 * CT_NSLOT + 6, bars + 2 * CT_NSLOT + 8, bars + 2 * CT_NSLOT + 10, bars + 2 * CT_NSLOT + 12};
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + CT_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CT_OFF_MISC + 4);
+  int* nunion_s = reinterpret_cast<int*>(sm + CT_OFF_MISC + 8);
+  int* cnt = reinterpret_cast<int*>(sm + CT_OFF_CNT);
+  int* ofs = reinterpret_cast<int*>(sm + CT_OFF_OFS);
+  uint32_t* uni = reinterpret_cast<uint32_t*>(sm + CT_OFF_UNI);
+  uint16_t* ent = reinterpret_cast<uint16_t*>(sm + CT_OFF_ENT);
+  float* Mw = reinterpret_cast<float*>(sm + CT_OFF_MW);
+  float* iZ = reinterpret_cast<float*>(sm + CT_OFF_IZ);
+  float* Ww = reinterpret_cast<float*>(sm + CT_OFF_WW);
+  int* posv = reinterpret_cast<int*>(sm + CT_OFF_POS);
+  int* part = reinterpret_cast<int*>(sm + CT_OFF_PART);
+
+  // ---------------------------------------------------------------- set-up
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_s, 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int j = 0; j < CT_NSLOT; ++j) { tc::mbar_init(&B.full[j], 1); tc::mbar_init(&B.empty[j], 1); }
+    for (int j = 0; j < 2; ++j) {
+      tc::mbar_init(&B.afull[j], 1);
+      tc::mbar_init(&B.aempty[j], 1);
+      tc::mbar_init(&B.sfull[j], 1);
+      tc::mbar_init(&B.sempty[j], 4);
+      tc::mbar_init(&B.pfull[j], 4);
+      tc::mbar_init(&B.pempty[j], 1);
+    }
+    tc::mbar_init(B.done, 1);
+    tc::mbar_fence_init();
+    *abort_flag = 0;
+  }
+  for (int q = tid; q < CT_TQ; q += CT_THREADS) {
+    const int i = i0 + q;
+    int p = INT_MIN;
+    if (i < Lq) {
+      const int pp = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+      if (!is_mask_slot(pp)) p = pp;
+    }
+    posv[q] = p;
+  }
+  for (int c = tid; c < C; c += CT_THREADS) cnt[c] = 0;
+  __syncthreads();
+  const int32_t* idx_t = idx + ((size_t)(b * Hkv + g) * Lq + i0) * K;
+  auto entry_chunk = [&](int e) -> int {     // chunk of (row e / K, slot e % K), -1 if none
+    const int q = e / K;
+    if (posv[q] == INT_MIN) return -1;
+    const int c = idx_t[e];
+    if (c < 0) return -1;
+    if (c >= C || !chunk_eligible(c, posv[q], w)) {
+      if (flags & RDL_FLAG_CHECKS) record_status(RDL_ERR_DEVICE_CHECK);
+      if (c >= C) return -1;
+    }
+    return c;
+  };
+  const int nent = min(CT_TQ, Lq - i0) * K;
+  for (int e = tid; e < nent; e += CT_THREADS) {
+    const int c = entry_chunk(e);
+    if (c >= 0) atomicAdd(&cnt[c], 1);
+  }
+  __syncthreads();
+  // exclusive scans of counts (entry offsets) and of non-empty flags (union slots)
+  {
+    const int per = (C + CT_THREADS - 1) / CT_THREADS, c0 = tid * per, c1 = min(C, c0 + per);
+    int s0 = 0, s1 = 0;
+    for (int c = c0; c < c1; ++c) { s0 += cnt[c]; s1 += cnt[c] > 0; }
+    part[2 * tid] = s0;
+    part[2 * tid + 1] = s1;
+    __syncthreads();
+    if (tid == 0) {
+      int a0 = 0, a1 = 0;
+      for (int t = 0; t < CT_THREADS; ++t) {
+        const int v0 = part[2 * t], v1 = part[2 * t + 1];
+        part[2 * t] = a0;
+        part[2 * t + 1] = a1;
+        a0 += v0;
+        a1 += v1;
+      }
+      *nunion_s = a1;
+    }
+    __syncthreads();
+    int r0 = part[2 * tid], r1 = part[2 * tid + 1];
+    for (int c = c0; c < c1; ++c) {
+      const int n = cnt[c];
+      ofs[c] = r0;
+      if (n > 0) uni[r1++] = ct_union(c, r0, n);
+      r0 += n;
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += CT_THREADS) cnt[c] = 0;     // becomes the scatter cursor
+  __syncthreads();
+  for (int e = tid; e < nent; e += CT_THREADS) {
+    const int c = entry_chunk(e);
+    if (c >= 0) {
+      const int pos = atomicAdd(&cnt[c], 1);
+      ent[ofs[c] + pos] = (uint16_t)(((e / K) << 8) | (e % K));
+    }
+  }
+  // fixed partition per (row, head): M = max(window planes, z), Z = sum of exponentials
+  const size_t plane_l = (size_t)gridDim.y / Hkv * Hq * Lq;
+  for (int e = tid; e < CT_TQ * G; e += CT_THREADS) {
+    const int q = e / G, h = e % G, i = i0 + q;
+    if (posv[q] == INT_MIN) continue;
+    const size_t li = (size_t)(b * Hq + g * G + h) * Lq + i;
+    const float* zr = z_sel + li * K;
+    float M = -INFINITY;
+    for (int s0 = 0; s0 < K; s0 += 8) {         // 8 independent loads per step
+      float zz[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) M = fmaxf(M, zz[u]);
+    }
+    for (int sw = 0; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
+    if (M == -INFINITY) M = 0.f;
+    float Z = 0.f;
+    for (int s0 = 0; s0 < K; s0 += 8) {
+      float zz[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) Z += expf(zz[u] - M);
+    }
+    float ls1 = -INFINITY;
+    for (int sw = 0; sw < nsw; ++sw) {
+      const float ls = lam_loc[sw * plane_l + li];
+      if (ls != -INFINITY) Z += expf(ls - M);
+      if (sw == 0) ls1 = ls;
+    }
+    Mw[q * 8 + h] = M;
+    iZ[q * 8 + h] = Z > 0.f ? 1.f / Z : 0.f;
+    // mass of the (single-plane) window part, used by the epilogue
+    Ww[q * 8 + h] = (nsw == 1 && ls1 != -INFINITY && Z > 0.f) ? expf(ls1 - M) / Z : 0.f;
+    if (lse) lse[li] = Z > 0.f ? M + logf(Z) : -INFINITY;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_s;
+  const int U = *nunion_s;
+  // zero the home accumulators
+  if (warp >= 2) {
+    const int qw = warp & 3;
+    const float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c0 = 0; c0 < CT_HOME; c0 += 8) tc::tmem_st8(tc::taddr(tbase, 32 * qw, c0), z8);
+    tc::tmem_wait_st();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+
+  const uint32_t smem_base = smem_u32(sm);
+  const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
+  const uint32_t idesc_pv = tc::idesc_bf16(128, 8, true, false);
+  // base descriptors (slot / buffer 0): Q rows and K are K-major, V^T is MN-major, P K-major
+  const uint64_t dA0 = tc::sdesc(smem_base + CT_OFF_A, 16, 1024);
+  const uint64_t dK0 = tc::sdesc(smem_base + CT_OFF_KV, 16, 1024);
+  const uint64_t dV0 = tc::sdesc(smem_base + CT_OFF_KV + 16384, 8192, 1024);
+  const uint64_t dP0 = tc::sdesc(smem_base + CT_OFF_P, 16, 1024);
+
+  // ---------------------------------------------------------------- producer
+  if (warp == 0) {
+    if (lane == 0) {
+      int k = 0;
+      for (int u = 0; u < U && !*abort_flag; ++u) {
+        const uint32_t un = uni[u];
+        const int c = un & 4095, start = (un >> 12) & 4095, n = un >> 24;
+        const int slot = u % CT_NSLOT;
+        if (!ct_wait(&B.empty[slot], ((u / CT_NSLOT) & 1) ^ 1, abort_flag)) break;
+        unsigned char* kv = sm + CT_OFF_KV + slot * 32768;
+        tc::mbar_arrive_expect_tx(&B.full[slot], 32768);
+        const int krow = (b * Hkv + g) * L + c * S;
+        tc::tma_load_2d(kv, &map_k, 0, krow, &B.full[slot]);
+        tc::tma_load_2d(kv + 8192, &map_k, 64, krow, &B.full[slot]);
+        tc::tma_load_2d(kv + 16384, &map_v, 0, krow, &B.full[slot]);
+        tc::tma_load_2d(kv + 24576, &map_v, 64, krow, &B.full[slot]);
+        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+          const int nq = min(CT_QP, n - p0), ab = k & 1;
+          if (!ct_wait(&B.aempty[ab], ((k >> 1) & 1) ^ 1, abort_flag)) break;
+          unsigned char* at = sm + CT_OFF_A + ab * 16384;
+          tc::mbar_arrive_expect_tx(&B.afull[ab], nq * 2048);
+          for (int j = 0; j < nq; ++j) {
+            const int ql = ent[start + p0 + j] >> 8;
+            const int qrow = ((b * Lq + i0 + ql) * Hq + g * G);
+            tc::tma_load_2d(at + j * 1024, &map_q, 0, qrow, &B.afull[ab]);
+            tc::tma_load_2d(at + 8192 + j * 1024, &map_q, 64, qrow, &B.afull[ab]);
+          }
+        }
+      }
+    }
+  }
+  // ---------------------------------------------------------------- MMA issuer
+  else if (warp == 1) {
+    if (lane == 0) {
+      int k = 0;
+      int pu = -1, pp0 = 0, pk = -1;     // previous item (chunk index, first query, item no.)
+      auto issue_pv = [&](int u, int p0, int kk) -> bool {
+        const uint32_t un = uni[u];
+        const int start = (un >> 12) & 4095, n = un >> 24;
+        const int nq = min(CT_QP, n - p0), pb = kk & 1, slot = u % CT_NSLOT;
+        if (!ct_wait(&B.pfull[pb], (kk >> 1) & 1, abort_flag)) return false;
+        tc::tc_fence_after();
+        // descriptors: the start-address field is the low 14 bits (address >> 4) and never
+        // carries, so offsets are added to a base descriptor
+        const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
+        const uint64_t bd0 = dP0 + (uint64_t)((pb * 8192) >> 4);
+        for (int j = 0; j < nq; ++j) {
+          const uint32_t dcol = tbase + (uint32_t)((ent[start + p0 + j] >> 8) * CT_HP);
+          const uint64_t bdj = bd0 + (uint64_t)(j * 64);
+          tc::mma_bf16_ss(dcol, ad0, bdj, idesc_pv, true);
+          tc::mma_bf16_ss(dcol, ad0 + 128, bdj + 2, idesc_pv, true);
+          tc::mma_bf16_ss(dcol, ad0 + 256, bdj + 4, idesc_pv, true);
+          tc::mma_bf16_ss(dcol, ad0 + 384, bdj + 6, idesc_pv, true);
+        }
+        tc::mma_commit(&B.pempty[pb]);
+        if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);   // last pass of this chunk
+        return true;
+      };
+      bool ok = true;
+      for (int u = 0; u < U && ok; ++u) {
+        const uint32_t un = uni[u];
+        const int n = un >> 24, slot = u % CT_NSLOT;
+        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) { ok = false; break; }
+        for (int p0 = 0; p0 < n && ok; p0 += CT_QP, ++k) {
+          const int ab = k & 1, sb = k & 1;
+          if (!ct_wait(&B.afull[ab], (k >> 1) & 1, abort_flag) ||
+              !ct_wait(&B.sempty[sb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint64_t da = dA0 + (uint64_t)((ab * 16384) >> 4);
+          const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
+          const uint32_t dS = tbase + (uint32_t)(CT_SCOL + 64 * sb);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);   // (bytes) >> 4
+            tc::mma_bf16_ss(dS, da + koff, dk + koff, idesc_s, ks > 0);
+          }
+          tc::mma_commit(&B.sfull[sb]);
+          tc::mma_commit(&B.aempty[ab]);
+          if (pk >= 0 && !issue_pv(pu, pp0, pk)) { ok = false; break; }
+          pu = u; pp0 = p0; pk = k;
+        }
+      }
+      if (ok && pk >= 0) issue_pv(pu, pp0, pk);
+      if (pk >= 0) tc::mma_commit(B.done);     // arrives once every issued MMA completed
+      else tc::mbar_arrive(B.done);
+    }
+  }
+  // ---------------------------------------------------------------- softmax warps
+  else {
+    const int qw = warp & 3;                       // TMEM lane quarter of this warp
+    const float sl2 = rsqrtf(128.f) * LOG2E;
+    const int r = 16 * qw + lane, jq = r >> 3, hh = r & 7;   // this thread's S row
+    // (row, slot) weight of the thread's row in a pass, fetched one pass ahead
+    auto pass_weight = [&](int start, int n, int p0) -> float {
+      const int nq = min(CT_QP, n - p0);
+      if (!(lane < 16 && jq < nq && hh < G)) return 0.f;
+      const uint16_t en = ent[start + p0 + jq];
+      const int ql = en >> 8, slot = en & 255;
+      const float zz = z_sel[((size_t)(b * Hq + g * G + hh) * Lq + i0 + ql) * K + slot];
+      return expf(zz - Mw[ql * 8 + hh]) * iZ[ql * 8 + hh];
+    };
+    int k = 0;
+    bool ok = true;
+    int nu = 0, np0 = 0;                           // next pass
+    float wnext = 0.f;
+    if (U > 0) wnext = pass_weight((uni[0] >> 12) & 4095, uni[0] >> 24, 0);
+    for (int u = 0; u < U && ok; ++u) {
+      const uint32_t un = uni[u];
+      const int start = (un >> 12) & 4095, n = un >> 24, c = un & 4095;
+      for (int p0 = 0; p0 < n && ok; p0 += CT_QP, ++k) {
+        const int sb = k & 1, pb = k & 1, nq = min(CT_QP, n - p0);
+        const float wcur = wnext;
+        // look ahead to the next pass and start its weight load now
+        np0 = p0 + CT_QP;
+        nu = u;
+        if (np0 >= n) { nu = u + 1; np0 = 0; }
+        if (nu < U) wnext = pass_weight((uni[nu] >> 12) & 4095, uni[nu] >> 24, np0);
+        if (!ct_wait(&B.sfull[sb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc::tc_fence_after();
+        float sv[64];
+        const uint32_t sa = tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * sb);
+        tc::tmem_ld16(sa, sv);
+        tc::tmem_ld16(sa + 16, sv + 16);
+        tc::tmem_ld16(sa + 32, sv + 32);
+        tc::tmem_ld16(sa + 48, sv + 48);
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&B.sempty[sb]);
+        // this thread's S row: r = 16*qw + lane (lanes 0..15), query slot r/8, head r%8
+        const bool valid = lane < 16 && jq < nq && hh < G;
+        const float scale = wcur;
+        float mx = -INFINITY;
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 63; ++j) mx = fmaxf(mx, sv[j]);
+        }
+        float l = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float pj = (valid && j < 63) ? fast_exp2((sv[j] - mx) * sl2) : 0.f;
+          sv[j] = pj;
+          l += pj;
+        }
+        const float f = (valid && l > 0.f) ? scale / l : 0.f;
+        if (!ct_wait(&B.pempty[pb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (lane < 16) {
+          unsigned char* prow = sm + CT_OFF_P + pb * 8192;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 v;
+            v.x = pack_bf16(sv[8 * ch] * f, sv[8 * ch + 1] * f);
+            v.y = pack_bf16(sv[8 * ch + 2] * f, sv[8 * ch + 3] * f);
+            v.z = pack_bf16(sv[8 * ch + 4] * f, sv[8 * ch + 5] * f);
+            v.w = pack_bf16(sv[8 * ch + 6] * f, sv[8 * ch + 7] * f);
+            *reinterpret_cast<uint4*>(prow + tc::sw128(r, 8 * ch)) = v;
+          }
+        }
+        tc::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&B.pfull[pb]);
+        (void)c;
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && ct_wait(B.done, 0, abort_flag)) {
+      tc::tc_fence_after();
+      const int d = 32 * qw + lane;                  // head-dim row held by this thread
+      const size_t plane = (size_t)gridDim.y / Hkv * Lq * Hq * 128;
+      for (int q = 0; q < CT_TQ; ++q) {
+        const int i = i0 + q;
+        if (i >= Lq) break;
+        float acc[8];
+        tc::tmem_ld8(tc::taddr(tbase, 32 * qw, q * CT_HP), acc);
+        tc::tmem_wait_ld();
+        if (posv[q] == INT_MIN) continue;
+        // each warp writes its 32 head-dim elements of every head: 64 contiguous bytes
+        __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + g * G) * 128;
+        const float* olr = o_loc + ((size_t)(b * Lq + i) * Hq + g * G) * 128 + d;
+        if (nsw == 1) {
+          float ol[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) ol[e2] = e2 < G ? olr[e2 * 128] : 0.f;
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2)
+            if (e2 < G) orow[e2 * 128 + d] = __float2bfloat16_rn(acc[e2] + Ww[q * 8 + e2] * ol[e2]);
+        } else {
+          for (int e2 = 0; e2 < G; ++e2) {
+            const size_t li = (size_t)(b * Hq + g * G + e2) * Lq + i;
+            float v = acc[e2];
+            for (int sw = 0; sw < nsw; ++sw) {
+              const float ls = lam_loc[sw * plane_l + li];
+              if (ls != -INFINITY) v += expf(ls - Mw[q * 8 + e2]) * iZ[q * 8 + e2] * olr[sw * plane + e2 * 128];
+            }
+            orow[e2 * 128 + d] = __float2bfloat16_rn(v);
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace rdl

@@ -277,3 +277,284 @@ __global__ void __launch_bounds__(128) topk_kernel(const float* __restrict__ zet
 }
 
 }  // namespace rdl
+
+namespace rdl {
+
+// --------------------------------------------------------------------------- radix top-K
+// Order-preserving map float -> uint32 (larger float, larger key; -inf lowest finite-less).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One warp per (b, g, i): exact top-K of zeta over the row by a 4-pass 8-bit radix select
+// for the K-th largest key, then one in-order pass that takes every key above it and the
+// first (by chunk index) of the keys equal to it -- ties to the smaller chunk index, and
+// the selection comes out in ascending chunk order.  Then the per-head scores of the
+// selected chunks are gathered.
+__global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict__ zeta,
+                                                         const float* __restrict__ z_all,
+                                                         const int32_t* __restrict__ q_pos, int Lq,
+                                                         int L, int Hq, int Hkv, int K,
+                                                         int32_t* __restrict__ idx,
+                                                         float* __restrict__ z_sel) {
+  extern __shared__ uint32_t tk_smem[];
+  const int C = L / S, G = Hq / Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long item = (long long)blockIdx.x * (blockDim.x / 32) + warp;
+  if (item >= (long long)Lq * Hkv) return;
+  const int b = blockIdx.y;
+  const int g = (int)(item / Lq), i = (int)(item % Lq);
+  uint32_t* keys = tk_smem + (size_t)warp * (C + 256);
+  uint32_t* hist = keys + C;
+  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+  int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
+  if (is_mask_slot(p)) {
+    for (int k = lane; k < K; k += 32) {
+      irow[k] = -1;
+      for (int hl = 0; hl < G; ++hl) z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
+    }
+    return;
+  }
+  const float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
+  const uint32_t kneg = order_key(-INFINITY);
+  int nvalid = 0;
+  int c = lane;
+  for (; c + 7 * 32 < C; c += 8 * 32) {      // 8 independent loads in flight per lane
+    float zv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) zv[u] = zr[c + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t k = order_key(zv[u]);
+      keys[c + 32 * u] = k;
+      nvalid += (k > kneg);
+    }
+  }
+  for (; c < C; c += 32) {
+    const uint32_t k = order_key(zr[c]);
+    keys[c] = k;
+    nvalid += (k > kneg);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
+  __syncwarp();
+  uint32_t thr = kneg;     // take keys > thr, plus `need` keys == thr (smallest indices)
+  int need = 0;
+  if (nvalid > K) {
+    uint32_t prefix = 0, pmask = 0;
+    need = K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0;
+      __syncwarp();
+      // scores cluster in a few digits (same sign/exponent): aggregate lanes that hit the
+      // same bin so each bin takes one atomic per step
+      for (int base = 0; base < C; base += 32) {
+        const int c = base + lane;
+        const uint32_t k = c < C ? keys[c] : 0u;
+        const bool in = c < C && (k & pmask) == prefix;
+        const unsigned dig = in ? ((k >> shift) & 255u) : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, dig);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+      }
+      __syncwarp();
+      // lane owns bins [8*lane, 8*lane+8); count of matching keys in bins above each lane
+      int local = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) local += (int)hist[lane * 8 + u];
+      // walk the lanes from the top bin down to the lane holding the need-th key
+      int incl = 0, target_lane = -1, excl_at_target = 0;
+      for (int l2 = 31; l2 >= 0; --l2) {
+        const int v = __shfl_sync(0xffffffffu, local, l2);
+        if (target_lane < 0 && incl + v >= need) { target_lane = l2; excl_at_target = incl; }
+        incl += v;
+      }
+      int digit = 0, cnt_above = excl_at_target;
+      if (lane == target_lane) {
+        int run = excl_at_target;
+        for (int u = 7; u >= 0; --u) {
+          const int v = (int)hist[lane * 8 + u];
+          if (run + v >= need) { digit = lane * 8 + u; cnt_above = run; break; }
+          run += v;
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, target_lane);
+      cnt_above = __shfl_sync(0xffffffffu, cnt_above, target_lane);
+      need -= cnt_above;
+      prefix |= (uint32_t)digit << shift;
+      pmask |= 255u << shift;
+      __syncwarp();
+    }
+    thr = prefix;
+  }
+  // in-order selection
+  int taken = 0, ties = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < C; base += 32) {
+    const int c = base + lane;
+    const uint32_t k = c < C ? keys[c] : 0u;
+    const bool tie = c < C && need > 0 && k == thr;
+    const unsigned tmask = __ballot_sync(0xffffffffu, tie);
+    const bool take = (c < C && k > thr) || (tie && ties + __popc(tmask & lt) < need);
+    ties += __popc(tmask);
+    const unsigned smask = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int pos = taken + __popc(smask & lt);
+      if (pos < K) irow[pos] = c;
+    }
+    taken += __popc(smask);
+  }
+  for (int k = taken + lane; k < K; k += 32) irow[k] = -1;
+  __syncwarp();
+  const int nsel = taken < K ? taken : K;
+  for (int e = lane; e < K * G; e += 32) {
+    const int k = e % K, hl = e / K, h = g * G + hl;
+    const int c = (k < nsel) ? irow[k] : -1;
+    z_sel[((size_t)(b * Hq + h) * Lq + i) * K + k] =
+        (c >= 0) ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
+  }
+}
+
+}  // namespace rdl
+
+namespace rdl {
+
+// Block-wide exclusive scan of one int per thread (256 threads); returns the total.
+__device__ __forceinline__ int block_excl_scan256(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < 8; ++w8) {
+    const int ws = warp_sums[w8];
+    if (w8 < warp) base += ws;
+    tot += ws;
+  }
+  __syncthreads();
+  total = tot;
+  return base + x - v;
+}
+
+// One CTA (256 threads) per (b, g, i): the same exact top-K as topk_radix_kernel, for few
+// rows over many chunks (decode blocks).  Keys are split across the CTA; the selection is
+// compacted in chunk order with block scans.
+__global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ zeta,
+                                                       const float* __restrict__ z_all,
+                                                       const int32_t* __restrict__ q_pos, int Lq, int L,
+                                                       int Hq, int Hkv, int K, int32_t* __restrict__ idx,
+                                                       float* __restrict__ z_sel) {
+  extern __shared__ uint32_t tc_keys[];
+  __shared__ unsigned hist[256];
+  __shared__ int warp_sums[8];
+  __shared__ int sel_s[64];
+  __shared__ int bc[3];
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int item = blockIdx.x, b = blockIdx.y;
+  const int g = item / Lq, i = item % Lq;
+  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+  int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
+  if (is_mask_slot(p)) {
+    for (int e = tid; e < K * G; e += 256) {
+      const int k = e % K, hl = e / K;
+      if (hl == 0) irow[k] = -1;
+      z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
+    }
+    return;
+  }
+  const float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
+  const uint32_t kneg = order_key(-INFINITY);
+  int nv = 0;
+  for (int c = tid; c < C; c += 256) {
+    const uint32_t k = order_key(zr[c]);
+    tc_keys[c] = k;
+    nv += k > kneg;
+  }
+  int nvalid;
+  (void)block_excl_scan256(nv, warp_sums, nvalid);
+  uint32_t thr = kneg;
+  int need = 0;
+  if (nvalid > K) {
+    uint32_t prefix = 0, pmask = 0;
+    need = K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      hist[tid] = 0;
+      __syncthreads();
+      for (int base = 0; base < C; base += 256) {
+        const int c = base + tid;
+        const uint32_t k = c < C ? tc_keys[c] : 0u;
+        const bool in = c < C && (k & pmask) == prefix;
+        const unsigned dig = in ? ((k >> shift) & 255u) : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, dig);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int local = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) local += (int)hist[lane * 8 + u];
+        int incl = 0, tl = -1, excl = 0;
+        for (int l2 = 31; l2 >= 0; --l2) {
+          const int v = __shfl_sync(0xffffffffu, local, l2);
+          if (tl < 0 && incl + v >= need) { tl = l2; excl = incl; }
+          incl += v;
+        }
+        if (lane == tl) {
+          int run = excl, dg = 0, ca = excl;
+          for (int u = 7; u >= 0; --u) {
+            const int v = (int)hist[lane * 8 + u];
+            if (run + v >= need) { dg = lane * 8 + u; ca = run; break; }
+            run += v;
+          }
+          bc[0] = dg;
+          bc[1] = ca;
+        }
+      }
+      __syncthreads();
+      need -= bc[1];
+      prefix |= (uint32_t)bc[0] << shift;
+      pmask |= 255u << shift;
+      __syncthreads();
+    }
+    thr = prefix;
+  }
+  // ordered compaction: thread t owns the contiguous range [t*seg, (t+1)*seg)
+  const int seg = (C + 255) / 256, c0 = tid * seg, c1 = min(C, c0 + seg);
+  int ngt = 0, nties = 0;
+  for (int c = c0; c < c1; ++c) {
+    const uint32_t k = tc_keys[c];
+    ngt += k > thr;
+    nties += (need > 0 && k == thr);
+  }
+  int tot;
+  const int tie_base = block_excl_scan256(nties, warp_sums, tot);
+  const int take_ties = max(0, min(nties, need - tie_base));
+  const int pos0 = block_excl_scan256(ngt + take_ties, warp_sums, tot);
+  int pos = pos0, tk = 0;
+  for (int c = c0; c < c1; ++c) {
+    const uint32_t k = tc_keys[c];
+    bool take = k > thr;
+    if (!take && need > 0 && k == thr && tk < take_ties) { take = true; ++tk; }
+    if (take && pos < K) sel_s[pos] = c;
+    pos += take;
+  }
+  __syncthreads();
+  const int nsel = min(tot, K);
+  for (int e = tid; e < K * G; e += 256) {
+    const int k = e % K, hl = e / K, h = g * G + hl;
+    const int c = k < nsel ? sel_s[k] : -1;
+    if (hl == 0) irow[k] = c;
+    z_sel[((size_t)(b * Hq + h) * Lq + i) * K + k] =
+        c >= 0 ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
+  }
+}
+
+}  // namespace rdl

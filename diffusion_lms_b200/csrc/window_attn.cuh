@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(128) generic_attn_kernel(
 // --------------------------------------------------------------------------- mma window
 // MODE 0: sliding-window layer output (o bf16, lse).  MODE 1: route-layer local window,
 // normalised o_loc (fp32) and its log-sum-exp lambda_loc, consumed by the chunk kernel.
+// With nsplit > 1 (few query rows, e.g. decode blocks) the key blocks of a row tile are
+// split over blockIdx.z and each split writes its own normalised output and log-sum-exp
+// to o_loc / lam_loc plane `split`; the chunk kernel (route) or window_combine_kernel
+// (sliding window) merges the planes.
 constexpr int WIN_ROWS = 16;
 constexpr int WIN_KEYS = 64;
 
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int L, int Lq,
     int Hq, int Hkv, int w, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-    float* __restrict__ o_loc, float* __restrict__ lam_loc) {
+    float* __restrict__ o_loc, float* __restrict__ lam_loc, int nsplit) {
   constexpr int D = 128;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char* Ks = smem_raw;                       // [2][64 rows][256 B]
@@ -166,7 +170,10 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
   }
   __syncthreads();
   const int kbeg = range_s[0], kend = range_s[1];
-  const int nblk = kend > kbeg ? (kend - kbeg + WIN_KEYS - 1) / WIN_KEYS : 0;
+  const int nblk_all = kend > kbeg ? (kend - kbeg + WIN_KEYS - 1) / WIN_KEYS : 0;
+  const int split = blockIdx.z;
+  const int per = (nblk_all + nsplit - 1) / nsplit;
+  const int blo = min(nblk_all, split * per), bhi = min(nblk_all, blo + per);
   const __nv_bfloat16* kg = k + (size_t)(b * Hkv + g) * L * D;
   const __nv_bfloat16* vg = v + (size_t)(b * Hkv + g) * L * D;
 
@@ -179,7 +186,7 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
       cp_async16(smem_u32(Vs + stage * WIN_KEYS * 256 + swz256(r, ch)), vg + (size_t)j * D + ch * 8);
     }
   };
-  if (nblk > 0) load_block(0, 0);
+  if (bhi > blo) load_block(blo, 0);
   cp_async_commit();
 
   const int gq = lane >> 2, tq = lane & 3;
@@ -193,13 +200,13 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
   uint32_t qa[8][4];
   const float sl2 = rsqrtf((float)D) * LOG2E;
 
-  for (int blk = 0; blk < nblk; ++blk) {
-    const int stage = blk & 1;
-    if (blk + 1 < nblk) load_block(blk + 1, stage ^ 1);
+  for (int blk = blo; blk < bhi; ++blk) {
+    const int stage = (blk - blo) & 1;
+    if (blk + 1 < bhi) load_block(blk + 1, stage ^ 1);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
-    if (blk == 0 && active) {
+    if (blk == blo && active) {
       const unsigned char* qw = Qs + warp * WIN_ROWS * 256;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
@@ -289,7 +296,11 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
   }
   cp_async_wait<0>();
   if (!active) return;
-  // epilogue: normalise and store
+  // epilogue: normalise and store (to the split's partial plane when there are splits)
+  const bool partial = (MODE == 1) || nsplit > 1;
+  const size_t plane = (size_t)gridDim.y / Hkv * Lq * Hq * D, plane_l = (size_t)gridDim.y / Hkv * Hq * Lq;
+  float* o_part = o_loc ? o_loc + (size_t)split * plane : nullptr;
+  float* l_part = lam_loc ? lam_loc + (size_t)split * plane_l : nullptr;
   const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
   const float ls0 = l0 > 0.f ? (m0 + __log2f(l0)) * LN2 : -INFINITY;
   const float ls1 = l1 > 0.f ? (m1 + __log2f(l1)) * LN2 : -INFINITY;
@@ -303,23 +314,53 @@ __global__ void __launch_bounds__(256) window_mma_kernel(
     for (int dn = 0; dn < 16; ++dn) {
       const int d0 = dn * 8 + 2 * tq;
       const float x0 = oacc[dn][2 * half] * inv, x1 = oacc[dn][2 * half + 1] * inv;
-      if (MODE == 0) {
+      if (!partial) {
         *reinterpret_cast<uint32_t*>(o + rowoff + d0) = pack_bf16(x0, x1);
       } else {
-        *reinterpret_cast<float2*>(o_loc + rowoff + d0) = make_float2(x0, x1);
+        *reinterpret_cast<float2*>(o_part + rowoff + d0) = make_float2(x0, x1);
       }
     }
     if (tq == 0) {
       const float ls = half ? ls1 : ls0;
-      if (MODE == 0) {
+      if (!partial) {
         if (lse) lse[(size_t)(b * Hq + h) * Lq + i] = ls;
       } else {
-        lam_loc[(size_t)(b * Hq + h) * Lq + i] = ls;
+        l_part[(size_t)(b * Hq + h) * Lq + i] = ls;
       }
     }
   }
 }
 
 inline size_t window_mma_smem(int G) { return (size_t)(4 * WIN_KEYS * 256 + G * WIN_ROWS * 256); }
+
+// Sliding-window output from key-split partials: lse = LSE_s lse_s, o = sum_s e^{lse_s-lse} o_s.
+// One thread per (row, head, element).
+__global__ void window_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ l_part,
+                                      int nsplit, int B, int Lq, int Hq, __nv_bfloat16* __restrict__ o,
+                                      float* __restrict__ lse) {
+  constexpr int D = 128;
+  const long long n = (long long)B * Lq * Hq * D;
+  const size_t plane = (size_t)n, plane_l = (size_t)B * Hq * Lq;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long rowh = e / D;                 // (b, i, h)
+    const int h = (int)(rowh % Hq);
+    const long long bi = rowh / Hq;
+    const int i = (int)(bi % Lq), b = (int)(bi / Lq);
+    const size_t li = (size_t)(b * Hq + h) * Lq + i;
+    float mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, l_part[s * plane_l + li]);
+    float z = 0.f, acc = 0.f;
+    if (mx != -INFINITY) {
+      for (int s = 0; s < nsplit; ++s) {
+        const float ls = l_part[s * plane_l + li];
+        const float wgt = (ls == -INFINITY) ? 0.f : expf(ls - mx);
+        z += wgt;
+        acc = fmaf(wgt, o_part[s * plane + e], acc);
+      }
+    }
+    o[e] = __float2bfloat16_rn(z > 0.f ? acc / z : 0.f);
+    if (lse && (e % D) == 0) lse[li] = z > 0.f ? mx + logf(z) : -INFINITY;
+  }
+}
 
 }  // namespace rdl

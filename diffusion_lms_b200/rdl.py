@@ -27,7 +27,7 @@ ERR_SCRATCH_LIMIT = -7
 NOALLOC_SCRATCH_BYTES = 16 << 20
 BF16, F32 = 0, 1
 FLAG_MEAN_SUMMARY, FLAG_CHECKS = 0x1, 0x2
-WS_SCORE, WS_ATTN = 0, 1
+WS_SCORE, WS_ATTN, WS_SWA = 0, 1, 2
 CHUNK = 64
 
 
@@ -52,7 +52,7 @@ _SIGS = {
                                     _sz, _vp]),
     "rdl_route_attn": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp, _sz, _vp]),
     "rdl_route_attn_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp]),
-    "rdl_swa_attn": (_int, [_vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp]),
+    "rdl_swa_attn": (_int, [_vp, _vp, _vp, _vp, _P, _int, _vp, _vp, _vp, _sz, _vp]),
     "rdl_workspace_bytes": (_sz, [_int, _P, _int]),
     "rdl_last_device_status": (_int, [_vp]),
     "rdl_status_string": (ctypes.c_char_p, [_int]),
@@ -182,10 +182,12 @@ def rdl_route_attn_noalloc(q, q_pos, k, v, idx, z_sel, dims: Dims, dtype, o, lse
     return _check("rdl_route_attn_noalloc", s, raise_on_error)
 
 
-def rdl_swa_attn(q, q_pos, k, v, dims: Dims, dtype, o, lse=None, stream=None,
-                 raise_on_error=True) -> int:
+def rdl_swa_attn(q, q_pos, k, v, dims: Dims, dtype, o, lse=None, workspace=None,
+                 ws_bytes: Optional[int] = None, stream=None, raise_on_error=True) -> int:
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     s = _lib.rdl_swa_attn(_p(q), _p(q_pos), _p(k), _p(v), ctypes.byref(dims.c()), _dt(dtype),
-                          _p(o), _p(lse), _stream(stream))
+                          _p(o), _p(lse), _p(workspace), ws_bytes, _stream(stream))
     return _check("rdl_swa_attn", s, raise_on_error)
 
 

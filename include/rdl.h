@@ -86,6 +86,7 @@ typedef struct {
 /* Which workspace a call needs (rdl_workspace_bytes). */
 #define RDL_WS_SCORE 0
 #define RDL_WS_ATTN 1
+#define RDL_WS_SWA 2
 
 /*
  * rdl_summary_pool -- summary key, pooling entropy and mask-slot output of every chunk
@@ -166,7 +167,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * Scratch limit: RDL_NOALLOC_SCRATCH_BYTES (16 MiB) per device, reserved on every GPU
  * that loads the library, until the process exits.  A call whose
  * rdl_workspace_bytes(RDL_WS_ATTN, dims, dtype) exceeds it returns RDL_ERR_SCRATCH_LIMIT
- * and launches nothing (a 32-query decode block over 28 heads needs about 4.2 MiB).
+ * and launches nothing (a 32-query decode block over 28 heads needs about 11.5 MiB).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture begins.
  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
@@ -186,10 +187,13 @@ rdl_status rdl_route_attn_noalloc(const void* q, const int32_t* q_pos, const voi
  * abstract; radius per Table 3).  Every row, mask slots included:
  *   o = softmax_{j in W(p)} (tau q.k_j) applied to v_j,   lse = LSE (nullable).
  * Requires w >= 0.  K, D, r, lambda are ignored.
+ * workspace (nullable): rdl_workspace_bytes(RDL_WS_SWA, dims, dtype) bytes, 256-byte
+ *   aligned.  It is nonzero only for few query rows (decode blocks), where the window's
+ *   keys are split across CTAs; with NULL the unsplit (slower for few rows) path runs.
  */
 rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, const void* v,
                         const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse,
-                        void* stream);
+                        void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes a call needs (0 if none); 0 also for invalid dims. */
 size_t rdl_workspace_bytes(int which, const rdl_dims* dims, rdl_dtype dtype);
