@@ -9,17 +9,23 @@
 //   bucketed by chunk (counting sort in shared memory).  For every chunk in the union, in
 //   ascending order, the K/V slab (2 x 16 KB) arrives by TMA, and the rows that selected it
 //   are processed 8 queries (64 rows = 8 x 8 padded heads) at a time:
-//     S   = Q_rows K_c^T        tcgen05.mma M=64 N=64 K=128 -> TMEM (double-buffered)
+//     S   = Q_rows K_c^T        tcgen05.mma M=64 N=64 K=128 -> TMEM buffer (k mod 2)
 //     P   = e^{S - max} * w_{i,h,c} / l   over the 63 content keys, written to smem (bf16)
-//     O^T[:, 8q..8q+8) += V_c^T P_q^T    tcgen05.mma M=128 (head dim) N=8 K=64, one per
-//                                         query, accumulating straight into that query's
-//                                         home columns of TMEM (no scatter pass)
+//     T   = V_c^T P^T               tcgen05.mma M=128 (head dim) N=8*nq K=64 -> the same
+//                                         TMEM buffer (S is in registers by then)
+//     O^T[:, 8q..8q+8) += T[:, 8j..8j+8)   lane-local TMEM adds into each query's home
+//                                         columns (one thread per head-dim lane)
 //   where w = e^{z_{i,h,c} - M}/Z is fixed up front (z_sel and the window lse are inputs).
 //   The home accumulators O^T [128 lanes x 48*8 columns] stay in TMEM for the whole tile;
 //   the epilogue adds the window part and writes o once.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (one thread) and
-// TMEM owner, warps 2-5 = softmax + epilogue (one per TMEM lane quarter).
+// Warp roles (480 threads): warp 0 = TMA producer, warp 1 = TMEM owner and issuer of the S
+// MMAs, warp 2 = issuer of the PV MMAs (small MMAs are issue-bound, so the two streams are
+// issued by different threads), warps 3-6 and 7-10 = two softmax groups taking even / odd
+// passes, warps 11-14 = home-column adds and the epilogue (each group has one warp per TMEM
+// lane quarter).  An M=64 result occupies lanes 0-15 of each quarter; the softmax reads it
+// with the 16x256b shape, which spreads 16 lanes over the 32 threads (thread t: rows t/4
+// and t/4+8, columns 8i + 2(t%4) + {0,1}), so every thread holds two rows x 16 columns.
 // Every wait is bounded; on a timeout the kernel records RDL_ERR_TIMEOUT, every role
 // stops, TMEM is freed and the kernel returns.
 #pragma once
@@ -35,15 +41,15 @@ constexpr int CT_NSLOT = 3;                // K/V ring depth
 constexpr int CT_MAXC = 2048;              // chunks (L <= 131072)
 constexpr int CT_MAXK = 64;
 constexpr int CT_HOME = CT_TQ * CT_HP;     // 384 home columns
-constexpr int CT_SCOL = CT_HOME;           // S buffers at 384 and 448
-constexpr int CT_THREADS = 192;
+constexpr int CT_SCOL = CT_HOME;           // S / PV buffers at 384..447 and 448..511
+constexpr int CT_THREADS = 480;
 
 // shared-memory map (bytes from the 1024-aligned base)
 constexpr int CT_OFF_KV = 0;                                   // slot s: K at s*32K, V at +16K
 constexpr int CT_OFF_A = CT_OFF_KV + CT_NSLOT * 32768;         // 2 x 16 KB gathered Q rows
 constexpr int CT_OFF_P = CT_OFF_A + 2 * 16384;                 // 2 x 8 KB P tiles
 constexpr int CT_OFF_BAR = CT_OFF_P + 2 * 8192;                // mbarriers
-constexpr int CT_NBAR = 2 * CT_NSLOT + 2 * 5 + 1;
+constexpr int CT_NBAR = 2 * CT_NSLOT + 16;
 constexpr int CT_OFF_MISC = CT_OFF_BAR + 256;                  // tmem base, abort, nunion
 constexpr int CT_OFF_CNT = CT_OFF_MISC + 128;                  // counts / cursor [MAXC] int
 constexpr int CT_OFF_OFS = CT_OFF_CNT + CT_MAXC * 4;           // offsets [MAXC] int
@@ -58,14 +64,15 @@ constexpr int CT_SMEM = CT_OFF_PART + CT_THREADS * 8 + 1024;   // + alignment sl
 
 struct CtBars {
   uint64_t* full;    // [NSLOT] K/V landed
-  uint64_t* empty;   // [NSLOT] K/V slot released (MMA commit)
+  uint64_t* empty;   // [NSLOT] K/V slot released (one commit from each MMA thread)
   uint64_t* afull;   // [2] gathered Q rows landed
-  uint64_t* aempty;  // [2] Q tile consumed by MMA1 (commit)
-  uint64_t* sfull;   // [2] S ready (commit)
-  uint64_t* sempty;  // [2] S read by the softmax warps (4 arrivals)
-  uint64_t* pfull;   // [2] P written (4 arrivals)
+  uint64_t* aempty;  // [2] Q tile consumed by the S MMAs (commit)
+  uint64_t* sfull;   // [2] S ready in TMEM buffer (commit)
+  uint64_t* pfull;   // [2] P written, S read out of its buffer (4 arrivals)
   uint64_t* pempty;  // [2] P consumed by the PV MMAs (commit)
-  uint64_t* done;    // all MMAs complete (commit)
+  uint64_t* tfull;   // [2] PV result ready in the buffer (commit)
+  uint64_t* tempty;  // [2] PV result added into the home columns: buffer free (4 arrivals)
+  uint64_t* done;    // [2] every MMA of the S / PV issuer complete (before TMEM is freed)
 };
 
 // bounded wait that also gives up as soon as another role has aborted
@@ -97,8 +104,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CT_OFF_BAR);
-  CtBars B{bars, bars + CT_NSLOT, bars + 2 * CT_NSLOT, bars + 2 * CT_NSLOT + 2, bars + 2 * CT_NSLOT + 4,
-           bars + 2 * CT_NSLOT + 6, bars + 2 * CT_NSLOT + 8, bars + 2 * CT_NSLOT + 10, bars + 2 * CT_NSLOT + 12};
+  uint64_t* b2 = bars + 2 * CT_NSLOT;
+  CtBars B{bars, bars + CT_NSLOT, b2, b2 + 2, b2 + 4, b2 + 6, b2 + 8, b2 + 10, b2 + 12, b2 + 14};
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + CT_OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CT_OFF_MISC + 4);
   int* nunion_s = reinterpret_cast<int*>(sm + CT_OFF_MISC + 8);
@@ -118,16 +125,17 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     tc::tmem_relinquish();
   }
   if (tid == 0) {
-    for (int j = 0; j < CT_NSLOT; ++j) { tc::mbar_init(&B.full[j], 1); tc::mbar_init(&B.empty[j], 1); }
+    for (int j = 0; j < CT_NSLOT; ++j) { tc::mbar_init(&B.full[j], 1); tc::mbar_init(&B.empty[j], 2); }
     for (int j = 0; j < 2; ++j) {
       tc::mbar_init(&B.afull[j], 1);
       tc::mbar_init(&B.aempty[j], 1);
       tc::mbar_init(&B.sfull[j], 1);
-      tc::mbar_init(&B.sempty[j], 4);
       tc::mbar_init(&B.pfull[j], 4);
       tc::mbar_init(&B.pempty[j], 1);
+      tc::mbar_init(&B.tfull[j], 1);
+      tc::mbar_init(&B.tempty[j], 4);
+      tc::mbar_init(&B.done[j], 1);
     }
-    tc::mbar_init(B.done, 1);
     tc::mbar_fence_init();
     *abort_flag = 0;
   }
@@ -241,7 +249,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   const uint32_t tbase = *tmem_s;
   const int U = *nunion_s;
   // zero the home accumulators
-  if (warp >= 2) {
+  if (warp >= 11) {
     const int qw = warp & 3;
     const float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int c0 = 0; c0 < CT_HOME; c0 += 8) tc::tmem_st8(tc::taddr(tbase, 32 * qw, c0), z8);
@@ -252,13 +260,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   tc::tc_fence_after();
 
   const uint32_t smem_base = smem_u32(sm);
-  const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
-  const uint32_t idesc_pv = tc::idesc_bf16(128, 8, true, false);
-  // base descriptors (slot / buffer 0): Q rows and K are K-major, V^T is MN-major, P K-major
+  // base descriptors (slot / buffer 0): Q rows and K are K-major, V^T is MN-major, P K-major.
+  // The start-address field is the low 14 bits (address >> 4) and never carries inside the
+  // shared window, so buffer / step offsets are added to these.
   const uint64_t dA0 = tc::sdesc(smem_base + CT_OFF_A, 16, 1024);
   const uint64_t dK0 = tc::sdesc(smem_base + CT_OFF_KV, 16, 1024);
   const uint64_t dV0 = tc::sdesc(smem_base + CT_OFF_KV + 16384, 8192, 1024);
   const uint64_t dP0 = tc::sdesc(smem_base + CT_OFF_P, 16, 1024);
+  // passes: chunk u of the union, queries p0 .. p0+7 of its bucket; pass k uses A, P and
+  // TMEM buffer k & 1
+  auto next_pass = [&](int& u, int& p0) {
+    p0 += CT_QP;
+    if (p0 >= (int)(uni[u] >> 24)) { ++u; p0 = 0; }
+  };
 
   // ---------------------------------------------------------------- producer
   if (warp == 0) {
@@ -291,162 +305,233 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
       }
     }
   }
-  // ---------------------------------------------------------------- MMA issuer
+  // ---------------------------------------------------------------- S MMAs
   else if (warp == 1) {
     if (lane == 0) {
+      const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
       int k = 0;
-      int pu = -1, pp0 = 0, pk = -1;     // previous item (chunk index, first query, item no.)
-      auto issue_pv = [&](int u, int p0, int kk) -> bool {
-        const uint32_t un = uni[u];
-        const int start = (un >> 12) & 4095, n = un >> 24;
-        const int nq = min(CT_QP, n - p0), pb = kk & 1, slot = u % CT_NSLOT;
-        if (!ct_wait(&B.pfull[pb], (kk >> 1) & 1, abort_flag)) return false;
-        tc::tc_fence_after();
-        // descriptors: the start-address field is the low 14 bits (address >> 4) and never
-        // carries, so offsets are added to a base descriptor
-        const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
-        const uint64_t bd0 = dP0 + (uint64_t)((pb * 8192) >> 4);
-        for (int j = 0; j < nq; ++j) {
-          const uint32_t dcol = tbase + (uint32_t)((ent[start + p0 + j] >> 8) * CT_HP);
-          const uint64_t bdj = bd0 + (uint64_t)(j * 64);
-          tc::mma_bf16_ss(dcol, ad0, bdj, idesc_pv, true);
-          tc::mma_bf16_ss(dcol, ad0 + 128, bdj + 2, idesc_pv, true);
-          tc::mma_bf16_ss(dcol, ad0 + 256, bdj + 4, idesc_pv, true);
-          tc::mma_bf16_ss(dcol, ad0 + 384, bdj + 6, idesc_pv, true);
-        }
-        tc::mma_commit(&B.pempty[pb]);
-        if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);   // last pass of this chunk
-        return true;
-      };
-      bool ok = true;
+      bool ok = true, issued = false;
       for (int u = 0; u < U && ok; ++u) {
-        const uint32_t un = uni[u];
-        const int n = un >> 24, slot = u % CT_NSLOT;
-        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) { ok = false; break; }
-        for (int p0 = 0; p0 < n && ok; p0 += CT_QP, ++k) {
-          const int ab = k & 1, sb = k & 1;
-          if (!ct_wait(&B.afull[ab], (k >> 1) & 1, abort_flag) ||
-              !ct_wait(&B.sempty[sb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        const int n = uni[u] >> 24, slot = u % CT_NSLOT;
+        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
+        const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
+        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+          const int bb = k & 1;
+          if (!ct_wait(&B.afull[bb], (k >> 1) & 1, abort_flag) ||
+              !ct_wait(&B.tempty[bb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint64_t da = dA0 + (uint64_t)((ab * 16384) >> 4);
-          const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
-          const uint32_t dS = tbase + (uint32_t)(CT_SCOL + 64 * sb);
+          const uint64_t da = dA0 + (uint64_t)((bb * 16384) >> 4);
+          const uint32_t dS = tbase + (uint32_t)(CT_SCOL + 64 * bb);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);   // (bytes) >> 4
+            const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);
             tc::mma_bf16_ss(dS, da + koff, dk + koff, idesc_s, ks > 0);
           }
-          tc::mma_commit(&B.sfull[sb]);
-          tc::mma_commit(&B.aempty[ab]);
-          if (pk >= 0 && !issue_pv(pu, pp0, pk)) { ok = false; break; }
-          pu = u; pp0 = p0; pk = k;
+          tc::mma_commit(&B.sfull[bb]);
+          tc::mma_commit(&B.aempty[bb]);
+          if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // K of this chunk done
+          issued = true;
         }
       }
-      if (ok && pk >= 0) issue_pv(pu, pp0, pk);
-      if (pk >= 0) tc::mma_commit(B.done);     // arrives once every issued MMA completed
-      else tc::mbar_arrive(B.done);
+      if (issued) tc::mma_commit(&B.done[0]); else tc::mbar_arrive(&B.done[0]);
+      tc::mbar_wait(&B.done[0], 0);          // bounded; not cut short by an abort
     }
   }
-  // ---------------------------------------------------------------- softmax warps
-  else {
+  // ---------------------------------------------------------------- PV MMAs
+  else if (warp == 2) {
+    if (lane == 0) {
+      int k = 0;
+      bool ok = true, issued = false;
+      for (int u = 0; u < U && ok; ++u) {
+        const int n = uni[u] >> 24, slot = u % CT_NSLOT;
+        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
+        const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
+        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+          const int nq = min(CT_QP, n - p0), bb = k & 1;
+          if (!ct_wait(&B.pfull[bb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint64_t bd0 = dP0 + (uint64_t)((bb * 8192) >> 4);
+          // N rounded up to a multiple of 16; P rows past 8*nq are zero
+          const uint32_t idesc_pv = tc::idesc_bf16(128, 16 * ((nq + 1) >> 1), true, false);
+          const uint32_t dT = tbase + (uint32_t)(CT_SCOL + 64 * bb);
+          tc::mma_bf16_ss(dT, ad0, bd0, idesc_pv, false);
+          tc::mma_bf16_ss(dT, ad0 + 128, bd0 + 2, idesc_pv, true);
+          tc::mma_bf16_ss(dT, ad0 + 256, bd0 + 4, idesc_pv, true);
+          tc::mma_bf16_ss(dT, ad0 + 384, bd0 + 6, idesc_pv, true);
+          tc::mma_commit(&B.tfull[bb]);
+          tc::mma_commit(&B.pempty[bb]);
+          if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // V of this chunk done
+          issued = true;
+        }
+      }
+      if (issued) tc::mma_commit(&B.done[1]); else tc::mbar_arrive(&B.done[1]);
+      tc::mbar_wait(&B.done[1], 0);
+    }
+  }
+  // ---------------------------------------------------------------- softmax groups
+  else if (warp <= 10) {
+    const int grp = (warp - 3) >> 2;               // passes k with k % 2 == grp
     const int qw = warp & 3;                       // TMEM lane quarter of this warp
     const float sl2 = rsqrtf(128.f) * LOG2E;
-    const int r = 16 * qw + lane, jq = r >> 3, hh = r & 7;   // this thread's S row
-    // (row, slot) weight of the thread's row in a pass, fetched one pass ahead
-    auto pass_weight = [&](int start, int n, int p0) -> float {
-      const int nq = min(CT_QP, n - p0);
-      if (!(lane < 16 && jq < nq && hh < G)) return 0.f;
-      const uint16_t en = ent[start + p0 + jq];
-      const int ql = en >> 8, slot = en & 255;
-      const float zz = z_sel[((size_t)(b * Hq + g * G + hh) * Lq + i0 + ql) * K + slot];
-      return expf(zz - Mw[ql * 8 + hh]) * iZ[ql * 8 + hh];
+    const int hh = lane >> 2, cq = 2 * (lane & 3);  // head row, column pair in each 8-group
+    const int jqa = 2 * qw, jqb = 2 * qw + 1;       // queries of rows 16qw + hh and +8
+    // per-row weight w = e^{z - M} / Z of a pass (raw z loaded one pass ahead)
+    struct RowW { float za, ma, iza, zb, mb, izb; };
+    auto pass_row = [&](int u, int p0) -> RowW {
+      RowW r{-INFINITY, 0.f, 0.f, -INFINITY, 0.f, 0.f};
+      if (u >= U || hh >= G) return r;
+      const uint32_t un = uni[u];
+      const int start = (un >> 12) & 4095, nq = min(CT_QP, (int)(un >> 24) - p0);
+      const float* zh = z_sel + ((size_t)(b * Hq + g * G + hh) * Lq + i0) * K;
+      if (jqa < nq) {
+        const uint16_t en = ent[start + p0 + jqa];
+        r.za = zh[(size_t)(en >> 8) * K + (en & 255)];
+        r.ma = Mw[(en >> 8) * 8 + hh];
+        r.iza = iZ[(en >> 8) * 8 + hh];
+      }
+      if (jqb < nq) {
+        const uint16_t en = ent[start + p0 + jqb];
+        r.zb = zh[(size_t)(en >> 8) * K + (en & 255)];
+        r.mb = Mw[(en >> 8) * 8 + hh];
+        r.izb = iZ[(en >> 8) * 8 + hh];
+      }
+      return r;
     };
+    int u = 0, p0 = 0, k = 0;
+    if (grp == 1 && U > 0) { next_pass(u, p0); k = 1; }
+    RowW wnext = pass_row(u, p0);
+    for (int m = 0; u < U; ++m) {
+      const int nq = min(CT_QP, (int)(uni[u] >> 24) - p0), bb = k & 1;
+      const RowW wc = wnext;
+      next_pass(u, p0);
+      if (u < U) next_pass(u, p0);                 // this group's next pass is k + 2
+      k += 2;
+      wnext = pass_row(u, p0);
+      if (!ct_wait(&B.sfull[bb], m & 1, abort_flag)) break;
+      tc::tc_fence_after();
+      float sv[32];
+      tc::tmem_ld16x256b_x8(tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * bb), sv);
+      tc::tmem_wait_ld();
+      const bool va = jqa < nq && hh < G, vb = jqb < nq && hh < G;
+      // sv[4i + 0,1]: row a, columns 8i + cq + {0,1}; sv[4i + 2,3]: row b, same columns.
+      // Column 63 (the routing-mask slot) is i = 7, cq = 6, second element.
+      const bool last = cq == 6;
+      float ma = fmaxf(sv[0], sv[1]), mb = fmaxf(sv[2], sv[3]);
+#pragma unroll
+      for (int i = 1; i < 8; ++i) {
+        ma = fmaxf(ma, (i == 7 && last) ? sv[4 * i] : fmaxf(sv[4 * i], sv[4 * i + 1]));
+        mb = fmaxf(mb, (i == 7 && last) ? sv[4 * i + 2] : fmaxf(sv[4 * i + 2], sv[4 * i + 3]));
+      }
+      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+      ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+      const float oa = va ? ma * sl2 : 0.f, ob = vb ? mb * sl2 : 0.f;
+      float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool mask1 = i == 7 && last;
+        sv[4 * i] = fast_exp2(fmaf(sv[4 * i], sl2, -oa));
+        sv[4 * i + 1] = mask1 ? 0.f : fast_exp2(fmaf(sv[4 * i + 1], sl2, -oa));
+        sv[4 * i + 2] = fast_exp2(fmaf(sv[4 * i + 2], sl2, -ob));
+        sv[4 * i + 3] = mask1 ? 0.f : fast_exp2(fmaf(sv[4 * i + 3], sl2, -ob));
+        la0 += sv[4 * i];
+        la1 += sv[4 * i + 1];
+        lb0 += sv[4 * i + 2];
+        lb1 += sv[4 * i + 3];
+      }
+      float la = la0 + la1, lb = lb0 + lb1;
+      la += __shfl_xor_sync(0xffffffffu, la, 1);
+      lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+      la += __shfl_xor_sync(0xffffffffu, la, 2);
+      lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+      const float fa = (va && la > 0.f) ? expf(wc.za - wc.ma) * wc.iza / la : 0.f;
+      const float fb = (vb && lb > 0.f) ? expf(wc.zb - wc.mb) * wc.izb / lb : 0.f;
+      if (!ct_wait(&B.pempty[bb], (m & 1) ^ 1, abort_flag)) break;
+      unsigned char* pt = sm + CT_OFF_P + bb * 8192;
+      const int ra = 16 * qw + hh, rb = ra + 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t wa = va ? pack_bf16(sv[4 * i] * fa, sv[4 * i + 1] * fa) : 0u;
+        const uint32_t wb = vb ? pack_bf16(sv[4 * i + 2] * fb, sv[4 * i + 3] * fb) : 0u;
+        *reinterpret_cast<uint32_t*>(pt + tc::sw128(ra, 8 * i + cq)) = wa;
+        *reinterpret_cast<uint32_t*>(pt + tc::sw128(rb, 8 * i + cq)) = wb;
+      }
+      tc::fence_proxy_async();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&B.pfull[bb]);
+    }
+  }
+  // ---------------------------------------------------------------- home adds + epilogue
+  else {
+    const int qw = warp & 3;
+    const int d = 32 * qw + lane;                  // head-dim row held by this thread
     int k = 0;
     bool ok = true;
-    int nu = 0, np0 = 0;                           // next pass
-    float wnext = 0.f;
-    if (U > 0) wnext = pass_weight((uni[0] >> 12) & 4095, uni[0] >> 24, 0);
     for (int u = 0; u < U && ok; ++u) {
       const uint32_t un = uni[u];
-      const int start = (un >> 12) & 4095, n = un >> 24, c = un & 4095;
+      const int start = (un >> 12) & 4095, n = un >> 24;
       for (int p0 = 0; p0 < n && ok; p0 += CT_QP, ++k) {
-        const int sb = k & 1, pb = k & 1, nq = min(CT_QP, n - p0);
-        const float wcur = wnext;
-        // look ahead to the next pass and start its weight load now
-        np0 = p0 + CT_QP;
-        nu = u;
-        if (np0 >= n) { nu = u + 1; np0 = 0; }
-        if (nu < U) wnext = pass_weight((uni[nu] >> 12) & 4095, uni[nu] >> 24, np0);
-        if (!ct_wait(&B.sfull[sb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int nq = min(CT_QP, n - p0), bb = k & 1;
+        if (!ct_wait(&B.tfull[bb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
         tc::tc_fence_after();
-        float sv[64];
-        const uint32_t sa = tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * sb);
-        tc::tmem_ld16(sa, sv);
-        tc::tmem_ld16(sa + 16, sv + 16);
-        tc::tmem_ld16(sa + 32, sv + 32);
-        tc::tmem_ld16(sa + 48, sv + 48);
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&B.sempty[sb]);
-        // this thread's S row: r = 16*qw + lane (lanes 0..15), query slot r/8, head r%8
-        const bool valid = lane < 16 && jq < nq && hh < G;
-        const float scale = wcur;
-        float mx = -INFINITY;
-        if (valid) {
+        const uint32_t tcol = tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * bb);
+        for (int j0 = 0; j0 < nq; j0 += 4) {        // 4 queries per round trip
+          float t8[4][8], h8[4][8];
+          int hc[4];
 #pragma unroll
-          for (int j = 0; j < 63; ++j) mx = fmaxf(mx, sv[j]);
-        }
-        float l = 0.f;
+          for (int j = 0; j < 4; ++j) {
+            if (j0 + j < nq) {
+              hc[j] = (ent[start + p0 + j0 + j] >> 8) * CT_HP;
+              tc::tmem_ld8(tcol + 8 * (j0 + j), t8[j]);
+              tc::tmem_ld8(tc::taddr(tbase, 32 * qw, hc[j]), h8[j]);
+            }
+          }
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float pj = (valid && j < 63) ? fast_exp2((sv[j] - mx) * sl2) : 0.f;
-          sv[j] = pj;
-          l += pj;
-        }
-        const float f = (valid && l > 0.f) ? scale / l : 0.f;
-        if (!ct_wait(&B.pempty[pb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (lane < 16) {
-          unsigned char* prow = sm + CT_OFF_P + pb * 8192;
+          for (int j = 0; j < 4; ++j) {
+            if (j0 + j < nq) {
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 v;
-            v.x = pack_bf16(sv[8 * ch] * f, sv[8 * ch + 1] * f);
-            v.y = pack_bf16(sv[8 * ch + 2] * f, sv[8 * ch + 3] * f);
-            v.z = pack_bf16(sv[8 * ch + 4] * f, sv[8 * ch + 5] * f);
-            v.w = pack_bf16(sv[8 * ch + 6] * f, sv[8 * ch + 7] * f);
-            *reinterpret_cast<uint4*>(prow + tc::sw128(r, 8 * ch)) = v;
+              for (int e2 = 0; e2 < 8; ++e2) h8[j][e2] += t8[j][e2];
+              tc::tmem_st8(tc::taddr(tbase, 32 * qw, hc[j]), h8[j]);
+            }
           }
         }
-        tc::fence_proxy_async();
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&B.pfull[pb]);
-        (void)c;
+        if (lane == 0) tc::mbar_arrive(&B.tempty[bb]);
       }
     }
-    // ------------------------------------------------------------ epilogue
-    if (ok && ct_wait(B.done, 0, abort_flag)) {
+    // epilogue: home columns + window part -> o (each warp writes its 32 head-dim lanes)
+    if (ok && !*abort_flag) {
       tc::tc_fence_after();
-      const int d = 32 * qw + lane;                  // head-dim row held by this thread
       const size_t plane = (size_t)gridDim.y / Hkv * Lq * Hq * 128;
-      for (int q = 0; q < CT_TQ; ++q) {
+      const int qn = min(CT_TQ, Lq - i0);
+      float olc[8], oln[8];
+      auto load_ol = [&](int q, float* ol) {
+        const float* olr = o_loc + ((size_t)(b * Lq + i0 + q) * Hq + g * G) * 128 + d;
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) ol[e2] = (nsw == 1 && e2 < G && posv[q] != INT_MIN) ? olr[e2 * 128] : 0.f;
+      };
+      if (qn > 0) load_ol(0, oln);
+      for (int q = 0; q < qn; ++q) {
         const int i = i0 + q;
-        if (i >= Lq) break;
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) olc[e2] = oln[e2];
+        if (q + 1 < qn) load_ol(q + 1, oln);
         float acc[8];
         tc::tmem_ld8(tc::taddr(tbase, 32 * qw, q * CT_HP), acc);
         tc::tmem_wait_ld();
         if (posv[q] == INT_MIN) continue;
-        // each warp writes its 32 head-dim elements of every head: 64 contiguous bytes
         __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + g * G) * 128;
-        const float* olr = o_loc + ((size_t)(b * Lq + i) * Hq + g * G) * 128 + d;
         if (nsw == 1) {
-          float ol[8];
-#pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) ol[e2] = e2 < G ? olr[e2 * 128] : 0.f;
 #pragma unroll
           for (int e2 = 0; e2 < 8; ++e2)
-            if (e2 < G) orow[e2 * 128 + d] = __float2bfloat16_rn(acc[e2] + Ww[q * 8 + e2] * ol[e2]);
+            if (e2 < G) orow[e2 * 128 + d] = __float2bfloat16_rn(acc[e2] + Ww[q * 8 + e2] * olc[e2]);
         } else {
+          const float* olr = o_loc + ((size_t)(b * Lq + i) * Hq + g * G) * 128 + d;
           for (int e2 = 0; e2 < G; ++e2) {
             const size_t li = (size_t)(b * Hq + g * G + e2) * Lq + i;
             float v = acc[e2];
