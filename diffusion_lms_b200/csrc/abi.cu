@@ -442,20 +442,20 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
   const int C = dims->L / S;
   if (ns == 1 && C <= CT_MAXC && dims->K <= CT_MAXK) {
     // prefill: tcgen05 kernel, 48-row tiles sharing each selected chunk's K/V
-    CUtensorMap mq, mk, mv;
-    const unsigned long long qrows = (unsigned long long)dims->B * dims->Lq * dims->Hq;
+    CtMaps maps;                                    // copied into the launch parameters
+    const unsigned long long tokens = (unsigned long long)dims->B * dims->Lq;
     const unsigned long long kvrows = (unsigned long long)dims->B * dims->Hkv * dims->L;
-    if (make_tmap_bf16(&mq, q, qrows, 128, 64, 8) && make_tmap_bf16(&mk, k, kvrows, 128, 64, 64) &&
-        make_tmap_bf16(&mv, v, kvrows, 128, 64, 64)) {
+    bool mapped = make_tmap_kv_halves(&maps.k, k, kvrows) && make_tmap_kv_halves(&maps.v, v, kvrows);
+    for (unsigned r = 1; r <= 8 && mapped; ++r) mapped = make_tmap_q_run(&maps.q[r - 1], q, tokens, dims->Hq, r);
+    if (mapped) {
       if (cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CT_SMEM) !=
           cudaSuccess)
         return RDL_ERR_CUDA;
       dim3 grid((dims->Lq + CT_TQ - 1) / CT_TQ, dims->B * dims->Hkv);
       count_launch();
-      chunk_tc_kernel<<<grid, CT_THREADS, CT_SMEM, st>>>(mq, mk, mv, q_pos, idx, z_sel, o_loc, lam_loc, nsw,
-                                                         dims->L, dims->Lq, dims->Hq, dims->Hkv, dims->K,
-                                                         dims->w, dims->flags, static_cast<__nv_bfloat16*>(o),
-                                                         lse);
+      chunk_tc_kernel<<<grid, CT_THREADS, CT_SMEM, st>>>(maps, q_pos, idx, z_sel, o_loc, lam_loc, nsw, dims->L,
+                                                         dims->Lq, dims->Hq, dims->Hkv, dims->K, dims->w,
+                                                         dims->flags, static_cast<__nv_bfloat16*>(o), lse);
       return cuda_status(cudaGetLastError());
     }
   }

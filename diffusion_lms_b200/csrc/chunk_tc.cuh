@@ -6,72 +6,101 @@
 // serves every query of a 48-row tile that selected it:
 //
 //   CTA = (48 consecutive query rows, one KV group).  The tile's (row, slot) selections are
-//   bucketed by chunk (counting sort in shared memory).  For every chunk in the union, in
-//   ascending order, the K/V slab (2 x 16 KB) arrives by TMA, and the rows that selected it
-//   are processed 8 queries (64 rows = 8 x 8 padded heads) at a time:
-//     S   = Q_rows K_c^T        tcgen05.mma M=64 N=64 K=128 -> TMEM buffer (k mod 2)
+//   bucketed by chunk, each bucket in ascending row order.  For every chunk in the union,
+//   in ascending order, the K/V slab (2 x 16 KB) arrives by TMA, and the rows that selected
+//   it are processed 8 queries (64 rows = 8 x 8 padded heads) at a time ("passes"):
+//     S   = Q_rows K_c^T        tcgen05.mma M=64 N=64 K=128 -> TMEM S region
 //     P   = e^{S - max} * w_{i,h,c} / l   over the 63 content keys, written to smem (bf16)
-//     T   = V_c^T P^T               tcgen05.mma M=128 (head dim) N=8*nq K=64 -> the same
-//                                         TMEM buffer (S is in registers by then)
+//     T   = V_c^T P^T           tcgen05.mma M=128 (head dim) N=8*nq K=64 -> TMEM T region
 //     O^T[:, 8q..8q+8) += T[:, 8j..8j+8)   lane-local TMEM adds into each query's home
 //                                         columns (one thread per head-dim lane)
 //   where w = e^{z_{i,h,c} - M}/Z is fixed up front (z_sel and the window lse are inputs).
 //   The home accumulators O^T [128 lanes x 48*8 columns] stay in TMEM for the whole tile;
 //   the epilogue adds the window part and writes o once.
 //
-// Warp roles (480 threads): warp 0 = TMA producer, warp 1 = TMEM owner and issuer of the S
-// MMAs, warp 2 = issuer of the PV MMAs (small MMAs are issue-bound, so the two streams are
-// issued by different threads), warps 3-6 and 7-10 = two softmax groups taking even / odd
-// passes, warps 11-14 = home-column adds and the epilogue (each group has one warp per TMEM
-// lane quarter).  An M=64 result occupies lanes 0-15 of each quarter; the softmax reads it
-// with the 16x256b shape, which spreads 16 lanes over the 32 threads (thread t: rows t/4
-// and t/4+8, columns 8i + 2(t%4) + {0,1}), so every thread holds two rows x 16 columns.
+// Costs that shape the design (measured on B200): a tcgen05.mma takes about the same issue
+// time (~50 cycles) for every shape up to N = 64, so a pass is bounded by its 12 MMAs; a
+// TMA instruction takes ~130 cycles to issue whatever its box size, so loads are made as
+// large as possible: K and V one 3D box each, and the Q rows of a pass one 4D box per run
+// of consecutive query tokens (the buckets are sorted so that runs are long).  S and T
+// have their own TMEM regions (S is released as soon as the softmax has read it), two
+// softmax groups take alternate passes, and the home adds are split over 8 warps.
+//
+// Warp roles (640 threads):
+//   warp 0        Q producer (TMA, lane 0)
+//   warp 1        TMEM owner, issuer of the S MMAs
+//   warp 2        issuer of the PV MMAs
+//   warps 3-10    two softmax groups (even / odd passes), one warp per TMEM lane quarter.
+//                 An M=64 result occupies lanes 0-15 of each quarter; the 16x256b load
+//                 shape spreads them over all 32 threads (thread t: rows t/4 and t/4+8,
+//                 columns 8i + 2(t%4) + {0,1}).
+//   warps 11-18   home-column adds (heads 0-3 / 4-7), then, with warps 3-10, the epilogue.
+//   warp 19       K/V producer (TMA, lane 0)
+// TMEM columns: home [0, 384), S [384, 448), T [448, 512).
+// Shared-memory Q tile of a pass: query slot j at j * 2 KB (columns 0-63 of its 8 head
+// rows, then columns 64-127), i.e. K-major with 128-byte swizzle, SBO 2 KB.
 // Every wait is bounded; on a timeout the kernel records RDL_ERR_TIMEOUT, every role
-// stops, TMEM is freed and the kernel returns.
+// stops, the MMAs in flight drain, TMEM is freed and the kernel returns.
 #pragma once
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace rdl {
 
-constexpr int CT_TQ = 48;                  // query rows per CTA
+constexpr int CT_TQ = 48;                  // query rows per CTA (<= 64: row masks)
 constexpr int CT_HP = 8;                   // rows per query in S / columns per query in TMEM
-constexpr int CT_QP = 8;                   // queries per MMA pass (M = 64)
+constexpr int CT_QP = 8;                   // queries per pass (M = 64)
 constexpr int CT_NSLOT = 3;                // K/V ring depth
+constexpr int CT_NA = 3;                   // Q ring depth
 constexpr int CT_MAXC = 2048;              // chunks (L <= 131072)
 constexpr int CT_MAXK = 64;
 constexpr int CT_HOME = CT_TQ * CT_HP;     // 384 home columns
-constexpr int CT_SCOL = CT_HOME;           // S / PV buffers at 384..447 and 448..511
-constexpr int CT_THREADS = 480;
+constexpr int CT_SCOL = CT_HOME;           // S region
+constexpr int CT_TCOL = CT_HOME + 64;      // T region
+constexpr int CT_WARPS = 20;
+constexpr int CT_THREADS = CT_WARPS * 32;
+constexpr int CT_EPI_THREADS = 16 * 32;    // warps 3-18
+constexpr int CT_KV_WARP = 19;
 
 // shared-memory map (bytes from the 1024-aligned base)
 constexpr int CT_OFF_KV = 0;                                   // slot s: K at s*32K, V at +16K
-constexpr int CT_OFF_A = CT_OFF_KV + CT_NSLOT * 32768;         // 2 x 16 KB gathered Q rows
-constexpr int CT_OFF_P = CT_OFF_A + 2 * 16384;                 // 2 x 8 KB P tiles
+constexpr int CT_OFF_A = CT_OFF_KV + CT_NSLOT * 32768;         // NA x 16 KB Q tiles
+constexpr int CT_OFF_P = CT_OFF_A + CT_NA * 16384;             // 2 x 8 KB P tiles
 constexpr int CT_OFF_BAR = CT_OFF_P + 2 * 8192;                // mbarriers
-constexpr int CT_NBAR = 2 * CT_NSLOT + 16;
+constexpr int CT_NBAR = 2 * CT_NSLOT + 2 * CT_NA + 11;
 constexpr int CT_OFF_MISC = CT_OFF_BAR + 256;                  // tmem base, abort, nunion
-constexpr int CT_OFF_CNT = CT_OFF_MISC + 128;                  // counts / cursor [MAXC] int
-constexpr int CT_OFF_OFS = CT_OFF_CNT + CT_MAXC * 4;           // offsets [MAXC] int
+constexpr int CT_OFF_MASK = CT_OFF_MISC + 128;                 // row masks [MAXC] u64
+constexpr int CT_OFF_OFS = CT_OFF_MASK + CT_MAXC * 8;          // bucket offsets [MAXC] int
 constexpr int CT_OFF_UNI = CT_OFF_OFS + CT_MAXC * 4;           // union [MAXC] u32
 constexpr int CT_OFF_ENT = CT_OFF_UNI + CT_MAXC * 4;           // entries [TQ*MAXK] u16
 constexpr int CT_OFF_MW = CT_OFF_ENT + CT_TQ * CT_MAXK * 2;    // M [TQ][8]
 constexpr int CT_OFF_IZ = CT_OFF_MW + CT_TQ * 8 * 4;           // 1/Z [TQ][8]
 constexpr int CT_OFF_WW = CT_OFF_IZ + CT_TQ * 8 * 4;           // window mass [TQ][8]
 constexpr int CT_OFF_POS = CT_OFF_WW + CT_TQ * 8 * 4;          // positions [TQ]
-constexpr int CT_OFF_PART = CT_OFF_POS + CT_TQ * 4;            // scan partials [192][2]
-constexpr int CT_SMEM = CT_OFF_PART + CT_THREADS * 8 + 1024;   // + alignment slack
+constexpr int CT_OFF_PART = CT_OFF_POS + CT_TQ * 4;            // scan partials [WARPS][2]
+constexpr int CT_SMEM = CT_OFF_PART + CT_WARPS * 8 + 1024;     // + alignment slack
+static_assert(CT_NBAR * 8 <= 256, "barrier area");
+static_assert(CT_SMEM <= 227 * 1024, "shared memory");
+static_assert(CT_TQ <= 64, "row masks are 64-bit");
+
+// Tensor maps of one launch: q as runs of 1..8 consecutive tokens (make_tmap_q_run), K and V
+// as 64-row slabs (make_tmap_kv_halves).
+struct CtMaps {
+  CUtensorMap q[8];
+  CUtensorMap k, v;
+};
 
 struct CtBars {
   uint64_t* full;    // [NSLOT] K/V landed
   uint64_t* empty;   // [NSLOT] K/V slot released (one commit from each MMA thread)
-  uint64_t* afull;   // [2] gathered Q rows landed
-  uint64_t* aempty;  // [2] Q tile consumed by the S MMAs (commit)
-  uint64_t* sfull;   // [2] S ready in TMEM buffer (commit)
-  uint64_t* pfull;   // [2] P written, S read out of its buffer (4 arrivals)
+  uint64_t* afull;   // [NA] Q tile landed
+  uint64_t* aempty;  // [NA] Q tile consumed by the S MMAs (commit)
+  uint64_t* sfull;   // [2] S of an even / odd pass ready (commit)
+  uint64_t* sempty;  // S region read by the softmax group of the pass (4 arrivals)
+  uint64_t* pfull;   // [2] P of an even / odd pass written (4 arrivals)
   uint64_t* pempty;  // [2] P consumed by the PV MMAs (commit)
-  uint64_t* tfull;   // [2] PV result ready in the buffer (commit)
-  uint64_t* tempty;  // [2] PV result added into the home columns: buffer free (4 arrivals)
+  uint64_t* tfull;   // T ready (commit)
+  uint64_t* tempty;  // T added into the home columns (8 arrivals)
   uint64_t* done;    // [2] every MMA of the S / PV issuer complete (before TMEM is freed)
 };
 
@@ -90,12 +119,15 @@ __device__ __forceinline__ uint32_t ct_union(int c, int start, int cnt) {
   return (uint32_t)c | ((uint32_t)start << 12) | ((uint32_t)cnt << 24);
 }
 
+__device__ __forceinline__ void ct_epi_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(CT_EPI_THREADS) : "memory");
+}
+
 __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
-    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-    const __grid_constant__ CUtensorMap map_v, const int32_t* __restrict__ q_pos,
-    const int32_t* __restrict__ idx, const float* __restrict__ z_sel, const float* __restrict__ o_loc,
-    const float* __restrict__ lam_loc, int nsw, int L, int Lq, int Hq, int Hkv, int K, int w, int flags,
-    __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    const __grid_constant__ CtMaps maps, const int32_t* __restrict__ q_pos, const int32_t* __restrict__ idx,
+    const float* __restrict__ z_sel, const float* __restrict__ o_loc, const float* __restrict__ lam_loc, int nsw,
+    int L, int Lq, int Hq, int Hkv, int K, int w, int flags, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ lse) {
   extern __shared__ unsigned char ct_raw[];
   unsigned char* sm = ct_raw + ((1024u - (smem_u32(ct_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -104,12 +136,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CT_OFF_BAR);
-  uint64_t* b2 = bars + 2 * CT_NSLOT;
-  CtBars B{bars, bars + CT_NSLOT, b2, b2 + 2, b2 + 4, b2 + 6, b2 + 8, b2 + 10, b2 + 12, b2 + 14};
+  uint64_t* b2 = bars + 2 * CT_NSLOT + 2 * CT_NA;
+  CtBars B{bars, bars + CT_NSLOT, bars + 2 * CT_NSLOT, bars + 2 * CT_NSLOT + CT_NA,
+           b2, b2 + 2, b2 + 3, b2 + 5, b2 + 7, b2 + 8, b2 + 9};
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + CT_OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CT_OFF_MISC + 4);
   int* nunion_s = reinterpret_cast<int*>(sm + CT_OFF_MISC + 8);
-  int* cnt = reinterpret_cast<int*>(sm + CT_OFF_CNT);
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(sm + CT_OFF_MASK);
   int* ofs = reinterpret_cast<int*>(sm + CT_OFF_OFS);
   uint32_t* uni = reinterpret_cast<uint32_t*>(sm + CT_OFF_UNI);
   uint16_t* ent = reinterpret_cast<uint16_t*>(sm + CT_OFF_ENT);
@@ -126,16 +159,16 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   }
   if (tid == 0) {
     for (int j = 0; j < CT_NSLOT; ++j) { tc::mbar_init(&B.full[j], 1); tc::mbar_init(&B.empty[j], 2); }
+    for (int j = 0; j < CT_NA; ++j) { tc::mbar_init(&B.afull[j], 1); tc::mbar_init(&B.aempty[j], 1); }
     for (int j = 0; j < 2; ++j) {
-      tc::mbar_init(&B.afull[j], 1);
-      tc::mbar_init(&B.aempty[j], 1);
       tc::mbar_init(&B.sfull[j], 1);
       tc::mbar_init(&B.pfull[j], 4);
       tc::mbar_init(&B.pempty[j], 1);
-      tc::mbar_init(&B.tfull[j], 1);
-      tc::mbar_init(&B.tempty[j], 4);
       tc::mbar_init(&B.done[j], 1);
     }
+    tc::mbar_init(B.sempty, 4);
+    tc::mbar_init(B.tfull, 1);
+    tc::mbar_init(B.tempty, 8);
     tc::mbar_fence_init();
     *abort_flag = 0;
   }
@@ -148,7 +181,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     }
     posv[q] = p;
   }
-  for (int c = tid; c < C; c += CT_THREADS) cnt[c] = 0;
+  for (int c = tid; c < C; c += CT_THREADS) mask[c] = 0ull;
   __syncthreads();
   const int32_t* idx_t = idx + ((size_t)(b * Hkv + g) * Lq + i0) * K;
   auto entry_chunk = [&](int e) -> int {     // chunk of (row e / K, slot e % K), -1 if none
@@ -162,48 +195,59 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     }
     return c;
   };
+  // bucket membership as row masks (a row selects a chunk at most once)
   const int nent = min(CT_TQ, Lq - i0) * K;
   for (int e = tid; e < nent; e += CT_THREADS) {
     const int c = entry_chunk(e);
-    if (c >= 0) atomicAdd(&cnt[c], 1);
+    if (c >= 0) atomicOr(&mask[c], 1ull << (e / K));
   }
   __syncthreads();
-  // exclusive scans of counts (entry offsets) and of non-empty flags (union slots)
+  // exclusive scans of bucket sizes (entry offsets) and of non-empty flags (union slots):
+  // per-thread runs of chunks, warp shuffles, then one warp over the warp totals
   {
     const int per = (C + CT_THREADS - 1) / CT_THREADS, c0 = tid * per, c1 = min(C, c0 + per);
-    int s0 = 0, s1 = 0;
-    for (int c = c0; c < c1; ++c) { s0 += cnt[c]; s1 += cnt[c] > 0; }
-    part[2 * tid] = s0;
-    part[2 * tid + 1] = s1;
+    int l0 = 0, l1 = 0;
+    for (int c = c0; c < c1; ++c) {
+      const int n = __popcll(mask[c]);
+      l0 += n;
+      l1 += n > 0;
+    }
+    int s0 = l0, s1 = l1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a0 = __shfl_up_sync(0xffffffffu, s0, off), a1 = __shfl_up_sync(0xffffffffu, s1, off);
+      if (lane >= off) { s0 += a0; s1 += a1; }
+    }
+    if (lane == 31) { part[2 * warp] = s0; part[2 * warp + 1] = s1; }
     __syncthreads();
-    if (tid == 0) {
-      int a0 = 0, a1 = 0;
-      for (int t = 0; t < CT_THREADS; ++t) {
-        const int v0 = part[2 * t], v1 = part[2 * t + 1];
-        part[2 * t] = a0;
-        part[2 * t + 1] = a1;
-        a0 += v0;
-        a1 += v1;
+    if (warp == 0) {
+      const int x0 = lane < CT_WARPS ? part[2 * lane] : 0, x1 = lane < CT_WARPS ? part[2 * lane + 1] : 0;
+      int y0 = x0, y1 = x1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int a0 = __shfl_up_sync(0xffffffffu, y0, off), a1 = __shfl_up_sync(0xffffffffu, y1, off);
+        if (lane >= off) { y0 += a0; y1 += a1; }
       }
-      *nunion_s = a1;
+      if (lane < CT_WARPS) { part[2 * lane] = y0 - x0; part[2 * lane + 1] = y1 - x1; }
+      if (lane == 31) *nunion_s = y1;
     }
     __syncthreads();
-    int r0 = part[2 * tid], r1 = part[2 * tid + 1];
+    int r0 = part[2 * warp] + s0 - l0, r1 = part[2 * warp + 1] + s1 - l1;
     for (int c = c0; c < c1; ++c) {
-      const int n = cnt[c];
+      const int n = __popcll(mask[c]);
       ofs[c] = r0;
       if (n > 0) uni[r1++] = ct_union(c, r0, n);
       r0 += n;
     }
   }
   __syncthreads();
-  for (int c = tid; c < C; c += CT_THREADS) cnt[c] = 0;     // becomes the scatter cursor
-  __syncthreads();
+  // entries in ascending row order inside each bucket: rank = rows below q in the mask
   for (int e = tid; e < nent; e += CT_THREADS) {
     const int c = entry_chunk(e);
     if (c >= 0) {
-      const int pos = atomicAdd(&cnt[c], 1);
-      ent[ofs[c] + pos] = (uint16_t)(((e / K) << 8) | (e % K));
+      const int q = e / K;
+      const int rank = __popcll(mask[c] & ((1ull << q) - 1ull));
+      ent[ofs[c] + rank] = (uint16_t)((q << 8) | (e % K));
     }
   }
   // fixed partition per (row, head): M = max(window planes, z), Z = sum of exponentials
@@ -213,23 +257,34 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     if (posv[q] == INT_MIN) continue;
     const size_t li = (size_t)(b * Hq + g * G + h) * Lq + i;
     const float* zr = z_sel + li * K;
-    float M = -INFINITY;
-    for (int s0 = 0; s0 < K; s0 += 8) {         // 8 independent loads per step
-      float zz[8];
+    float M = -INFINITY, Z = 0.f;
+    if (K <= 32) {                              // all loads in flight at once
+      float zz[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+      for (int u = 0; u < 32; ++u) zz[u] = u < K ? zr[u] : -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) M = fmaxf(M, zz[u]);
-    }
-    for (int sw = 0; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
-    if (M == -INFINITY) M = 0.f;
-    float Z = 0.f;
-    for (int s0 = 0; s0 < K; s0 += 8) {
-      float zz[8];
+      for (int u = 0; u < 32; ++u) M = fmaxf(M, zz[u]);
+      for (int sw = 0; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
+      if (M == -INFINITY) M = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+      for (int u = 0; u < 32; ++u) Z += expf(zz[u] - M);
+    } else {
+      for (int s0 = 0; s0 < K; s0 += 8) {
+        float zz[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) Z += expf(zz[u] - M);
+        for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) M = fmaxf(M, zz[u]);
+      }
+      for (int sw = 0; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
+      if (M == -INFINITY) M = 0.f;
+      for (int s0 = 0; s0 < K; s0 += 8) {
+        float zz[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) zz[u] = s0 + u < K ? zr[s0 + u] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) Z += expf(zz[u] - M);
+      }
     }
     float ls1 = -INFINITY;
     for (int sw = 0; sw < nsw; ++sw) {
@@ -249,7 +304,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   const uint32_t tbase = *tmem_s;
   const int U = *nunion_s;
   // zero the home accumulators
-  if (warp >= 11) {
+  if (warp >= 11 && warp < 15) {
     const int qw = warp & 3;
     const float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int c0 = 0; c0 < CT_HOME; c0 += 8) tc::tmem_st8(tc::taddr(tbase, 32 * qw, c0), z8);
@@ -263,45 +318,53 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   // base descriptors (slot / buffer 0): Q rows and K are K-major, V^T is MN-major, P K-major.
   // The start-address field is the low 14 bits (address >> 4) and never carries inside the
   // shared window, so buffer / step offsets are added to these.
-  const uint64_t dA0 = tc::sdesc(smem_base + CT_OFF_A, 16, 1024);
+  const uint64_t dA0 = tc::sdesc(smem_base + CT_OFF_A, 16, 2048);
   const uint64_t dK0 = tc::sdesc(smem_base + CT_OFF_KV, 16, 1024);
   const uint64_t dV0 = tc::sdesc(smem_base + CT_OFF_KV + 16384, 8192, 1024);
   const uint64_t dP0 = tc::sdesc(smem_base + CT_OFF_P, 16, 1024);
-  // passes: chunk u of the union, queries p0 .. p0+7 of its bucket; pass k uses A, P and
-  // TMEM buffer k & 1
+  // passes: chunk u of the union, queries p0 .. p0+7 of its bucket; pass k uses Q buffer
+  // k % NA and P buffer k & 1
   auto next_pass = [&](int& u, int& p0) {
     p0 += CT_QP;
     if (p0 >= (int)(uni[u] >> 24)) { ++u; p0 = 0; }
   };
 
-  // ---------------------------------------------------------------- producer
+  // ---------------------------------------------------------------- Q producer
   if (warp == 0) {
     if (lane == 0) {
       int k = 0;
-      for (int u = 0; u < U && !*abort_flag; ++u) {
+      bool ok = true;
+      for (int u = 0; u < U && ok; ++u) {
         const uint32_t un = uni[u];
-        const int c = un & 4095, start = (un >> 12) & 4095, n = un >> 24;
-        const int slot = u % CT_NSLOT;
+        const int start = (un >> 12) & 4095, n = un >> 24;
+        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+          const int nq = min(CT_QP, n - p0), ab = k % CT_NA;
+          if (!ct_wait(&B.aempty[ab], ((k / CT_NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          unsigned char* at = sm + CT_OFF_A + ab * 16384;
+          tc::mbar_arrive_expect_tx(&B.afull[ab], nq * 2048);
+          // one box per run of consecutive query tokens (bucket rows ascend)
+          for (int j = 0; j < nq;) {
+            const int ql = ent[start + p0 + j] >> 8;
+            int r = 1;
+            while (j + r < nq && (ent[start + p0 + j + r] >> 8) == ql + r) ++r;
+            tc::tma_load_4d(at + j * 2048, &maps.q[r - 1], 0, g * G, 0, b * Lq + i0 + ql, &B.afull[ab]);
+            j += r;
+          }
+        }
+      }
+    }
+  }
+  // ---------------------------------------------------------------- K/V producer
+  else if (warp == CT_KV_WARP) {
+    if (lane == 0) {
+      for (int u = 0; u < U; ++u) {
+        const int c = uni[u] & 4095, slot = u % CT_NSLOT;
         if (!ct_wait(&B.empty[slot], ((u / CT_NSLOT) & 1) ^ 1, abort_flag)) break;
         unsigned char* kv = sm + CT_OFF_KV + slot * 32768;
         tc::mbar_arrive_expect_tx(&B.full[slot], 32768);
         const int krow = (b * Hkv + g) * L + c * S;
-        tc::tma_load_2d(kv, &map_k, 0, krow, &B.full[slot]);
-        tc::tma_load_2d(kv + 8192, &map_k, 64, krow, &B.full[slot]);
-        tc::tma_load_2d(kv + 16384, &map_v, 0, krow, &B.full[slot]);
-        tc::tma_load_2d(kv + 24576, &map_v, 64, krow, &B.full[slot]);
-        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
-          const int nq = min(CT_QP, n - p0), ab = k & 1;
-          if (!ct_wait(&B.aempty[ab], ((k >> 1) & 1) ^ 1, abort_flag)) break;
-          unsigned char* at = sm + CT_OFF_A + ab * 16384;
-          tc::mbar_arrive_expect_tx(&B.afull[ab], nq * 2048);
-          for (int j = 0; j < nq; ++j) {
-            const int ql = ent[start + p0 + j] >> 8;
-            const int qrow = ((b * Lq + i0 + ql) * Hq + g * G);
-            tc::tma_load_2d(at + j * 1024, &map_q, 0, qrow, &B.afull[ab]);
-            tc::tma_load_2d(at + 8192 + j * 1024, &map_q, 64, qrow, &B.afull[ab]);
-          }
-        }
+        tc::tma_load_3d(kv, &maps.k, 0, krow, 0, &B.full[slot]);
+        tc::tma_load_3d(kv + 16384, &maps.v, 0, krow, 0, &B.full[slot]);
       }
     }
   }
@@ -309,6 +372,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
+      const uint32_t dS = tbase + (uint32_t)CT_SCOL;
       int k = 0;
       bool ok = true, issued = false;
       for (int u = 0; u < U && ok; ++u) {
@@ -316,19 +380,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
         if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
         const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
         for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
-          const int bb = k & 1;
-          if (!ct_wait(&B.afull[bb], (k >> 1) & 1, abort_flag) ||
-              !ct_wait(&B.tempty[bb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int ab = k % CT_NA, sb = k & 1;
+          if (!ct_wait(&B.afull[ab], (k / CT_NA) & 1, abort_flag) ||
+              !ct_wait(B.sempty, (k & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint64_t da = dA0 + (uint64_t)((bb * 16384) >> 4);
-          const uint32_t dS = tbase + (uint32_t)(CT_SCOL + 64 * bb);
+          const uint64_t da = dA0 + (uint64_t)((ab * 16384) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
+          for (int ks = 0; ks < 8; ++ks) {      // K steps of 16: halves at +1 KB (Q) / +8 KB (K)
+            const uint64_t qoff = (uint64_t)((ks >> 2) * 64 + (ks & 3) * 2);
             const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);
-            tc::mma_bf16_ss(dS, da + koff, dk + koff, idesc_s, ks > 0);
+            tc::mma_bf16_ss(dS, da + qoff, dk + koff, idesc_s, ks > 0);
           }
-          tc::mma_commit(&B.sfull[bb]);
-          tc::mma_commit(&B.aempty[bb]);
+          tc::mma_commit(&B.sfull[sb]);
+          tc::mma_commit(&B.aempty[ab]);
           if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // K of this chunk done
           issued = true;
         }
@@ -340,6 +404,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   // ---------------------------------------------------------------- PV MMAs
   else if (warp == 2) {
     if (lane == 0) {
+      const uint32_t dT = tbase + (uint32_t)CT_TCOL;
       int k = 0;
       bool ok = true, issued = false;
       for (int u = 0; u < U && ok; ++u) {
@@ -347,19 +412,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
         if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
         const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
         for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
-          const int nq = min(CT_QP, n - p0), bb = k & 1;
-          if (!ct_wait(&B.pfull[bb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+          const int nq = min(CT_QP, n - p0), pb = k & 1;
+          if (!ct_wait(&B.pfull[pb], (k >> 1) & 1, abort_flag) ||
+              !ct_wait(B.tempty, (k & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint64_t bd0 = dP0 + (uint64_t)((bb * 8192) >> 4);
+          const uint64_t bd0 = dP0 + (uint64_t)((pb * 8192) >> 4);
           // N rounded up to a multiple of 16; P rows past 8*nq are zero
           const uint32_t idesc_pv = tc::idesc_bf16(128, 16 * ((nq + 1) >> 1), true, false);
-          const uint32_t dT = tbase + (uint32_t)(CT_SCOL + 64 * bb);
           tc::mma_bf16_ss(dT, ad0, bd0, idesc_pv, false);
           tc::mma_bf16_ss(dT, ad0 + 128, bd0 + 2, idesc_pv, true);
           tc::mma_bf16_ss(dT, ad0 + 256, bd0 + 4, idesc_pv, true);
           tc::mma_bf16_ss(dT, ad0 + 384, bd0 + 6, idesc_pv, true);
-          tc::mma_commit(&B.tfull[bb]);
-          tc::mma_commit(&B.pempty[bb]);
+          tc::mma_commit(B.tfull);
+          tc::mma_commit(&B.pempty[pb]);
           if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // V of this chunk done
           issued = true;
         }
@@ -397,21 +462,23 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
       }
       return r;
     };
-    int u = 0, p0 = 0, k = 0;
-    if (grp == 1 && U > 0) { next_pass(u, p0); k = 1; }
+    int u = 0, p0 = 0;
+    if (grp == 1 && U > 0) next_pass(u, p0);
     RowW wnext = pass_row(u, p0);
     for (int m = 0; u < U; ++m) {
-      const int nq = min(CT_QP, (int)(uni[u] >> 24) - p0), bb = k & 1;
+      const int nq = min(CT_QP, (int)(uni[u] >> 24) - p0);
       const RowW wc = wnext;
       next_pass(u, p0);
-      if (u < U) next_pass(u, p0);                 // this group's next pass is k + 2
-      k += 2;
+      if (u < U) next_pass(u, p0);                 // this group's next pass
       wnext = pass_row(u, p0);
-      if (!ct_wait(&B.sfull[bb], m & 1, abort_flag)) break;
+      if (!ct_wait(&B.sfull[grp], m & 1, abort_flag)) break;
       tc::tc_fence_after();
       float sv[32];
-      tc::tmem_ld16x256b_x8(tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * bb), sv);
+      tc::tmem_ld16x256b_x8(tc::taddr(tbase, 32 * qw, CT_SCOL), sv);
       tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(B.sempty);    // S region free for the next pass
       const bool va = jqa < nq && hh < G, vb = jqb < nq && hh < G;
       // sv[4i + 0,1]: row a, columns 8i + cq + {0,1}; sv[4i + 2,3]: row b, same columns.
       // Column 63 (the routing-mask slot) is i = 7, cq = 6, second element.
@@ -447,8 +514,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
       lb += __shfl_xor_sync(0xffffffffu, lb, 2);
       const float fa = (va && la > 0.f) ? expf(wc.za - wc.ma) * wc.iza / la : 0.f;
       const float fb = (vb && lb > 0.f) ? expf(wc.zb - wc.mb) * wc.izb / lb : 0.f;
-      if (!ct_wait(&B.pempty[bb], (m & 1) ^ 1, abort_flag)) break;
-      unsigned char* pt = sm + CT_OFF_P + bb * 8192;
+      if (!ct_wait(&B.pempty[grp], (m & 1) ^ 1, abort_flag)) break;
+      unsigned char* pt = sm + CT_OFF_P + grp * 8192;
       const int ra = 16 * qw + hh, rb = ra + 8;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -458,90 +525,103 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
         *reinterpret_cast<uint32_t*>(pt + tc::sw128(rb, 8 * i + cq)) = wb;
       }
       tc::fence_proxy_async();
-      tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&B.pfull[bb]);
+      if (lane == 0) tc::mbar_arrive(&B.pfull[grp]);
     }
   }
-  // ---------------------------------------------------------------- home adds + epilogue
-  else {
+  // ---------------------------------------------------------------- home adds
+  else if (warp <= 18) {
     const int qw = warp & 3;
-    const int d = 32 * qw + lane;                  // head-dim row held by this thread
+    const int hs = 4 * ((warp - 11) >> 2);         // heads hs .. hs+3 of every query
+    const uint32_t lanebase = tc::taddr(tbase, 32 * qw, 0);
     int k = 0;
     bool ok = true;
     for (int u = 0; u < U && ok; ++u) {
       const uint32_t un = uni[u];
       const int start = (un >> 12) & 4095, n = un >> 24;
       for (int p0 = 0; p0 < n && ok; p0 += CT_QP, ++k) {
-        const int nq = min(CT_QP, n - p0), bb = k & 1;
-        if (!ct_wait(&B.tfull[bb], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int nq = min(CT_QP, n - p0);
+        // home column of query j of this pass, held by lane j
+        const int hcol = lane < nq ? (ent[start + p0 + lane] >> 8) * CT_HP + hs : 0;
+        if (!ct_wait(B.tfull, k & 1, abort_flag)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t tcol = tc::taddr(tbase, 32 * qw, CT_SCOL + 64 * bb);
-        for (int j0 = 0; j0 < nq; j0 += 4) {        // 4 queries per round trip
-          float t8[4][8], h8[4][8];
-          int hc[4];
+        if (hs < G) {
+          for (int j0 = 0; j0 < nq; j0 += 4) {      // 4 queries per round trip
+            float t4[4][4], h4[4][4];
+            int hc[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j0 + j < nq) {
-              hc[j] = (ent[start + p0 + j0 + j] >> 8) * CT_HP;
-              tc::tmem_ld8(tcol + 8 * (j0 + j), t8[j]);
-              tc::tmem_ld8(tc::taddr(tbase, 32 * qw, hc[j]), h8[j]);
+            for (int j = 0; j < 4; ++j) {
+              hc[j] = __shfl_sync(0xffffffffu, hcol, (j0 + j) & 31);
+              if (j0 + j < nq) {
+                tc::tmem_ld4(lanebase + (uint32_t)(CT_TCOL + 8 * (j0 + j) + hs), t4[j]);
+                tc::tmem_ld4(lanebase + (uint32_t)hc[j], h4[j]);
+              }
+            }
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (j0 + j < nq) {
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) h4[j][e2] += t4[j][e2];
+                tc::tmem_st4(lanebase + (uint32_t)hc[j], h4[j]);
+              }
             }
           }
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j0 + j < nq) {
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2) h8[j][e2] += t8[j][e2];
-              tc::tmem_st8(tc::taddr(tbase, 32 * qw, hc[j]), h8[j]);
-            }
-          }
+          tc::tmem_wait_st();
         }
-        tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&B.tempty[bb]);
+        if (lane == 0) tc::mbar_arrive(B.tempty);
       }
     }
-    // epilogue: home columns + window part -> o (each warp writes its 32 head-dim lanes)
-    if (ok && !*abort_flag) {
+  }
+  // ---------------------------------------------------------------- epilogue
+  // home columns + window part -> o; warps 3-18, four per TMEM lane quarter, take every
+  // fourth query (each warp writes its 32 head-dim lanes)
+  if (warp >= 3 && warp <= 18) {
+    ct_epi_sync();
+    if (!*abort_flag) {
       tc::tc_fence_after();
+      const int qw = warp & 3, e4 = (warp - 3) >> 2;
+      const int d = 32 * qw + lane;
       const size_t plane = (size_t)gridDim.y / Hkv * Lq * Hq * 128;
       const int qn = min(CT_TQ, Lq - i0);
-      float olc[8], oln[8];
       auto load_ol = [&](int q, float* ol) {
+        const bool on = nsw == 1 && q < qn && posv[q] != INT_MIN;
         const float* olr = o_loc + ((size_t)(b * Lq + i0 + q) * Hq + g * G) * 128 + d;
 #pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) ol[e2] = (nsw == 1 && e2 < G && posv[q] != INT_MIN) ? olr[e2 * 128] : 0.f;
+        for (int e2 = 0; e2 < 8; ++e2) ol[e2] = (on && e2 < G) ? olr[e2 * 128] : 0.f;
       };
-      if (qn > 0) load_ol(0, oln);
-      for (int q = 0; q < qn; ++q) {
-        const int i = i0 + q;
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) olc[e2] = oln[e2];
-        if (q + 1 < qn) load_ol(q + 1, oln);
+      float ol0[8], ol1[8], ol2[8];                // window rows of queries q, q+4, q+8
+      load_ol(e4, ol0);
+      load_ol(e4 + 4, ol1);
+      for (int q = e4; q < qn; q += 4) {
+        load_ol(q + 8, ol2);
         float acc[8];
         tc::tmem_ld8(tc::taddr(tbase, 32 * qw, q * CT_HP), acc);
         tc::tmem_wait_ld();
-        if (posv[q] == INT_MIN) continue;
-        __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + g * G) * 128;
-        if (nsw == 1) {
+        if (posv[q] != INT_MIN) {
+          const int i = i0 + q;
+          __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + g * G) * 128;
+          if (nsw == 1) {
 #pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2)
-            if (e2 < G) orow[e2 * 128 + d] = __float2bfloat16_rn(acc[e2] + Ww[q * 8 + e2] * olc[e2]);
-        } else {
-          const float* olr = o_loc + ((size_t)(b * Lq + i) * Hq + g * G) * 128 + d;
-          for (int e2 = 0; e2 < G; ++e2) {
-            const size_t li = (size_t)(b * Hq + g * G + e2) * Lq + i;
-            float v = acc[e2];
-            for (int sw = 0; sw < nsw; ++sw) {
-              const float ls = lam_loc[sw * plane_l + li];
-              if (ls != -INFINITY) v += expf(ls - Mw[q * 8 + e2]) * iZ[q * 8 + e2] * olr[sw * plane + e2 * 128];
+            for (int e2 = 0; e2 < 8; ++e2)
+              if (e2 < G) orow[e2 * 128 + d] = __float2bfloat16_rn(acc[e2] + Ww[q * 8 + e2] * ol0[e2]);
+          } else {
+            const float* olr = o_loc + ((size_t)(b * Lq + i) * Hq + g * G) * 128 + d;
+            for (int e2 = 0; e2 < G; ++e2) {
+              const size_t li = (size_t)(b * Hq + g * G + e2) * Lq + i;
+              float v = acc[e2];
+              for (int sw = 0; sw < nsw; ++sw) {
+                const float ls = lam_loc[sw * plane_l + li];
+                if (ls != -INFINITY) v += expf(ls - Mw[q * 8 + e2]) * iZ[q * 8 + e2] * olr[sw * plane + e2 * 128];
+              }
+              orow[e2 * 128 + d] = __float2bfloat16_rn(v);
             }
-            orow[e2 * 128 + d] = __float2bfloat16_rn(v);
           }
         }
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) { ol0[e2] = ol1[e2]; ol1[e2] = ol2[e2]; }
       }
     }
   }

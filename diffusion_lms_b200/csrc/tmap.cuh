@@ -38,4 +38,35 @@ inline bool make_tmap_bf16(CUtensorMap* map, const void* base, unsigned long lon
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K or V of one KV head as [rows x 128] bf16 (row stride 256 B), viewed as (64 columns,
+// rows, 2 halves) so that one box of 64 rows x 2 halves lands as two 8 KB 128-byte-swizzled
+// tiles (columns 0-63, then 64-127).
+inline bool make_tmap_kv_halves(CUtensorMap* map, const void* base, unsigned long long rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Queries q [tokens, Hq, 128] bf16 viewed as (64 columns, Hq heads, 2 halves, tokens): one box
+// of 8 heads x 2 halves x R consecutive tokens lands token-major, 2 KB per token (half 0 of
+// its 8 head rows, then half 1), each 1 KB a 128-byte-swizzled tile.  Heads past Hq read as 0.
+inline bool make_tmap_q_run(CUtensorMap* map, const void* base, unsigned long long tokens, unsigned Hq,
+                            unsigned run) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64, Hq, 2, tokens};
+  cuuint64_t strides[3] = {256, 128, (cuuint64_t)Hq * 256};
+  cuuint32_t box[4] = {64, 8, 2, run};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace rdl
