@@ -3,9 +3,9 @@
 // Same partition as chunk_mma_kernel ([v2] Figure 3 caption: the selected chunk scores and
 // the window's log-sum-exp share one softmax partition; a second softmax spreads each
 // chunk's mass over its 63 content tokens), organised so that one load of a chunk's K/V
-// serves every query of a 48-row tile that selected it:
+// serves every query of a 45-row tile that selected it:
 //
-//   CTA = (48 consecutive query rows, one KV group).  The tile's (row, slot) selections are
+//   CTA = (45 consecutive query rows, one KV group).  The tile's (row, slot) selections are
 //   bucketed by chunk, each bucket in ascending row order.  For every chunk in the union,
 //   in ascending order, the K/V slab (2 x 16 KB) arrives by TMA, and the rows that selected
 //   it are processed 8 queries (64 rows = 8 x 8 padded heads) at a time ("passes"):
@@ -15,7 +15,7 @@
 //     O^T[:, 8q..8q+8) += T[:, 8j..8j+8)   lane-local TMEM adds into each query's home
 //                                         columns (one thread per head-dim lane)
 //   where w = e^{z_{i,h,c} - M}/Z is fixed up front (z_sel and the window lse are inputs).
-//   The home accumulators O^T [128 lanes x 48*8 columns] stay in TMEM for the whole tile;
+//   The home accumulators O^T [128 lanes x 45*8 columns] stay in TMEM for the whole tile;
 //   the epilogue adds the window part and writes o once.
 //
 // Costs that shape the design (measured on B200): a tcgen05.mma takes about the same issue
@@ -36,7 +36,7 @@
 //                 columns 8i + 2(t%4) + {0,1}).
 //   warps 11-18   home-column adds (heads 0-3 / 4-7), then, with warps 3-10, the epilogue.
 //   warp 19       K/V producer (TMA, lane 0)
-// TMEM columns: home [0, 384), S [384, 448), T [448, 512).
+// TMEM columns: home [0, 360), S [384, 448), T [448, 512).
 // Shared-memory Q tile of a pass: query slot j at j * 2 KB (columns 0-63 of its 8 head
 // rows, then columns 64-127), i.e. K-major with 128-byte swizzle, SBO 2 KB.
 // Every wait is bounded; on a timeout the kernel records RDL_ERR_TIMEOUT, every role
@@ -47,16 +47,17 @@
 
 namespace rdl {
 
-constexpr int CT_TQ = 48;                  // query rows per CTA (<= 64: row masks)
+constexpr int CT_TQ = 45;                  // query rows per CTA (<= 64: row masks; 16K rows x 4 groups -> 9.9 waves of 148)
 constexpr int CT_HP = 8;                   // rows per query in S / columns per query in TMEM
 constexpr int CT_QP = 8;                   // queries per pass (M = 64)
 constexpr int CT_NSLOT = 3;                // K/V ring depth
 constexpr int CT_NA = 3;                   // Q ring depth
 constexpr int CT_MAXC = 2048;              // chunks (L <= 131072)
 constexpr int CT_MAXK = 64;
-constexpr int CT_HOME = CT_TQ * CT_HP;     // 384 home columns
-constexpr int CT_SCOL = CT_HOME;           // S region
-constexpr int CT_TCOL = CT_HOME + 64;      // T region
+constexpr int CT_HOME = CT_TQ * CT_HP;     // 360 home columns
+constexpr int CT_SCOL = 384;               // S region
+constexpr int CT_TCOL = 448;               // T region
+static_assert(CT_HOME <= CT_SCOL, "TMEM columns");
 constexpr int CT_WARPS = 20;
 constexpr int CT_THREADS = CT_WARPS * 32;
 constexpr int CT_EPI_THREADS = 16 * 32;    // warps 3-18
