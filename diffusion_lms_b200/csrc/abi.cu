@@ -16,6 +16,8 @@
 #include "chunk_attn.cuh"
 #include "tmap.cuh"
 #include "chunk_tc.cuh"
+#include "decode.cuh"
+#include <cstdlib>
 
 using namespace rdl;
 
@@ -86,6 +88,100 @@ bool fast_score(const rdl_dims* dm, rdl_dtype t) {
 }
 // decode blocks: few rows, head dim 128 -> the decode score path
 bool decode_score_path(const rdl_dims* dm) { return dm->d == 128 && dm->Lq <= 64; }
+
+// Decode blocks on the chained kernels of decode.cuh: bf16, head dim 128, at most 64 rows
+// per sequence, at most 8 heads per group, residual rank 0, 64 or 128.
+constexpr int kSMs = 148;
+bool dec_rows_ok(const rdl_dims* dm, rdl_dtype t) {
+  return t == RDL_BF16 && dm->d == 128 && dm->Lq <= 64 && dm->Hq / dm->Hkv <= 8;
+}
+bool dec_score_ok(const rdl_dims* dm, rdl_dtype t) {
+  return dec_rows_ok(dm, t) && dm->K <= kMaxK &&
+         (dm->r == 0 || ((dm->r == 64 || dm->r == 128) && dm->D % 64 == 0));
+}
+// decode attention (chunk-major, balanced): at most 32 rows and 2048 chunks per sequence,
+// at most 64 window slabs per row
+bool dec_attn_rows_ok(const rdl_dims* dm, rdl_dtype t) {
+  return t == RDL_BF16 && dm->d == 128 && dm->Lq <= dec::AT_QROWS && dm->Hq / dm->Hkv <= 8 &&
+         dm->L / S <= dec::AT_MAXC && dec::max_win_slabs(dm->w) <= 64;
+}
+bool dec_attn_ok(const rdl_dims* dm, rdl_dtype t) { return dec_attn_rows_ok(dm, t) && dm->K <= kMaxK; }
+bool dec_swa_ok(const rdl_dims* dm, rdl_dtype t) { return dec_attn_rows_ok(dm, t) && dm->w >= 0; }
+int dec_attn_stages(const rdl_dims* dm, int K) {
+  const int nwt = dec::max_win_slabs(dm->w);
+  for (int st = 4; st >= 2; --st)
+    if (dec::attn_smem(st, dm->Lq, K, dm->L / S, nwt).total <= 232448) return st;
+  return 0;
+}
+int dec_attn_ranges(const rdl_dims* dm) {
+  const int r = kSMs / (dm->B * dm->Hkv);
+  return r < 1 ? 1 : r;
+}
+// score grid: (ranges, Hq, B) with the range split into TMA boxes through a 3-stage ring
+struct DecScoreGrid {
+  int MT, ranges, ncr, boxr, nbox, nstg, smem;
+};
+DecScoreGrid dec_score_grid(const rdl_dims* dm) {
+  DecScoreGrid gr{};
+  const int C = dm->L / S;
+  gr.MT = dm->Lq <= 16 ? 1 : (dm->Lq <= 32 ? 2 : 4);
+  int ranges = kSMs / (dm->B * dm->Hq);
+  if (ranges < 1) ranges = 1;
+  int ncr = (C + ranges - 1) / ranges;
+  ncr = (ncr + 7) & ~7;
+  gr.ranges = (C + ncr - 1) / ncr;
+  gr.ncr = ncr;
+  // ring depth and box height: as many of the range's summary rows as fit in shared memory
+  // are loaded before the dependency wait
+  const int limit = 232448;
+  int best = -1;
+  for (int nstg = 4; nstg >= 2; --nstg) {
+    const int aux = dec::score_smem(gr.MT, dm->r, 0, nstg, ncr).total;
+    int boxr = ((limit - aux) / (nstg * 512)) & ~7;
+    if (boxr > 256) boxr = 256;
+    const int want = ((ncr + nstg - 1) / nstg + 7) & ~7;
+    if (boxr > want) boxr = want;
+    if (boxr < 8) continue;
+    const int pre = nstg * boxr < ncr ? nstg * boxr : ncr;
+    if (pre > best) {
+      best = pre;
+      gr.nstg = nstg;
+      gr.boxr = boxr;
+    }
+  }
+  gr.nbox = (ncr + gr.boxr - 1) / gr.boxr;
+  gr.smem = dec::score_smem(gr.MT, dm->r, gr.boxr, gr.nstg, ncr).total;
+  return gr;
+}
+bool use_pdl() {
+  static const bool on = [] {
+    const char* e = std::getenv("RDL_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+// Launch with programmatic dependent launch allowed (the kernel waits on its predecessor
+// with griddepcontrol.wait before touching anything the predecessor may write).
+template <typename... Exp, typename... Act>
+cudaError_t launch_ex(bool pdl, void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Act&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = (pdl && use_pdl()) ? 1 : 0;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+template <typename... Exp, typename... Act>
+cudaError_t launch_pdl(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Act&&... args) {
+  return launch_ex(true, kern, grid, block, smem, st, std::forward<Act>(args)...);
+}
 struct ScoreWs {
   size_t t, qres, z_all, zeta, tt, sb, tpart, total;
 };
@@ -94,8 +190,11 @@ ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   ScoreWs w{};
   size_t off = 0;
   w.z_all = off; off += align256(sizeof(float) * (size_t)dm->B * dm->Hq * dm->Lq * C);
-  w.zeta = off;  off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
-  if (fast_score(dm, dt)) {
+  w.zeta = off;
+  if (!dec_score_ok(dm, dt)) off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
+  if (dec_score_ok(dm, dt)) {
+    w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
+  } else if (fast_score(dm, dt)) {
     w.tt = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Lq * 2 * dm->r);
     w.sb = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Hq * C * (2 * dm->d + 2 * dm->r));
   } else {
@@ -115,6 +214,18 @@ struct AttnWs {
 AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
   AttnWs w{};
   if (!fast_attn(dm, t)) return w;
+  if (dec_attn_ok(dm, t) && dec_attn_stages(dm, dm->K) > 0) {
+    // chunk outputs [B, Lq, Hkv, K, G, d], window slab sums [B, Lq, Hkv, nwt, G, d] and
+    // their (max, sum) [B, Lq, Hkv, nwt, G]
+    const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
+    const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
+    size_t off = 0;
+    w.o_acc = off;   off += align256(sizeof(float) * rows * dm->K * dm->d);
+    w.o_loc = off;   off += align256(sizeof(float) * rows * nwt * dm->d);
+    w.lam_loc = off; off += align256(sizeof(float2) * rows * nwt);
+    w.total = off;
+    return w;
+  }
   const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
   size_t off = 0;
   const int nsw = window_splits(dm);
@@ -130,6 +241,11 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
 // Sliding-window workspace: key-split partials when the row count is small (else none).
 size_t swa_ws(const rdl_dims* dm, rdl_dtype t) {
   if (!fast_attn(dm, t) || dm->w < 0) return 0;
+  if (dec_swa_ok(dm, t) && dec_attn_stages(dm, 0) > 0) {
+    const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
+    const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
+    return align256(sizeof(float) * rows * nwt * dm->d) + align256(sizeof(float2) * rows * nwt);
+  }
   const int nsw = window_splits(dm);
   if (nsw <= 1) return 0;
   const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
@@ -171,6 +287,119 @@ rdl_status launch_topk(const float* zeta, const float* z_all, const int32_t* q_p
   topk_radix_kernel<<<g4, warps * 32, smem, st>>>(zeta, z_all, q_pos, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K,
                                                   idx, z_sel);
   return cuda_status(cudaGetLastError());
+}
+
+rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, const void* w_down,
+                        const void* w_up, const float* summary, const float* entropy, const rdl_dims* dm,
+                        int32_t* idx, float* z_sel, void* workspace, cudaStream_t st) {
+  const ScoreWs wl = score_ws(dm, RDL_BF16);
+  char* ws = static_cast<char*>(workspace);
+  float* t = reinterpret_cast<float*>(ws + wl.t);
+  float* z_all = reinterpret_cast<float*>(ws + wl.z_all);
+  const int C = dm->L / S, M = dm->B * dm->Lq;
+  const bool res = dm->r > 0 && x;
+  const DecScoreGrid gr = dec_score_grid(dm);
+  CUtensorMap smap;
+  if (!make_tmap_f32_rows(&smap, summary, (unsigned long long)dm->B * dm->Hq * C, (unsigned)gr.boxr))
+    return RDL_ERR_CUDA;
+  if (res) {
+    const int slice = ((dm->D + dec::TK_CL * 64 - 1) / (dec::TK_CL * 64)) * 64;
+    const int kc = slice < dec::TK_KMAX ? slice : dec::TK_KMAX;
+    const int rows = ((M + 15) / 16) * 16;
+    const int tsm = dec::tk_smem(rows, dm->r, kc);
+    CUtensorMap xmap, wmap;
+    if (!make_tmap_bf16(&xmap, x, (unsigned long long)M, (unsigned)dm->D, 64, (unsigned)rows) ||
+        !make_tmap_bf16(&wmap, w_down, (unsigned long long)dm->D, (unsigned)dm->r, 64, 64))
+      return RDL_ERR_CUDA;
+    if (cudaFuncSetAttribute(dec::dec_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    if (launch_pdl(dec::dec_t_kernel, dim3(dec::TK_CL), dim3(256), tsm, st, xmap, wmap, M, dm->D, dm->r, kc, t) !=
+        cudaSuccess)
+      return RDL_ERR_CUDA;
+  }
+  auto kern = gr.MT == 1 ? dec::dec_score_kernel<1> : (gr.MT == 2 ? dec::dec_score_kernel<2> : dec::dec_score_kernel<4>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gr.smem) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const float tau = (float)(1.0 / sqrt((double)dm->d));
+  // launched early only behind dec_t_kernel: its prologue loads inputs before the wait
+  if (launch_ex(res, kern, dim3(gr.ranges, dm->Hq, dm->B), dim3(256), gr.smem, st, smap, summary,
+                 static_cast<const __nv_bfloat16*>(q), q_pos, (const float*)(res ? t : nullptr),
+                 static_cast<const __nv_bfloat16*>(w_up), entropy, dm->Lq, dm->L, dm->Hq, res ? dm->r : 0, dm->w, tau,
+                 dm->lambda, gr.ncr, gr.boxr, gr.nbox, gr.nstg, z_all) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const int G = dm->Hq / dm->Hkv;
+  const bool zs = C % 4 == 0 && G * C <= dec::DK_MAXZ;
+  const size_t ksm = (size_t)(((C + 3) & ~3) + (zs ? G * C : 0)) * sizeof(uint32_t);
+  auto tk = C <= 1024 ? (zs ? dec::dec_topk_kernel<true, 4> : dec::dec_topk_kernel<false, 4>)
+            : C <= 2048 ? (zs ? dec::dec_topk_kernel<true, 8> : dec::dec_topk_kernel<false, 8>)
+                        : (zs ? dec::dec_topk_kernel<true, 32> : dec::dec_topk_kernel<false, 32>);
+  if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksm) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  if (launch_pdl(tk, dim3(dm->Lq, dm->Hkv, dm->B), dim3(256), ksm, st, (const float*)z_all, q_pos, dm->Lq, dm->L,
+                 dm->Hq, dm->Hkv, dm->K, idx, z_sel) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  return RDL_OK;
+}
+
+rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const void* v, const int32_t* idx,
+                       const float* z_sel, const rdl_dims* dm, void* o, float* lse, void* workspace,
+                       cudaStream_t st) {
+  const AttnWs wl = attn_ws(dm, RDL_BF16);
+  char* ws = static_cast<char*>(workspace);
+  float* o_part = reinterpret_cast<float*>(ws + wl.o_acc);
+  float* ow_part = reinterpret_cast<float*>(ws + wl.o_loc);
+  float2* ml_part = reinterpret_cast<float2*>(ws + wl.lam_loc);
+  const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
+  CUtensorMap kmap, vmap;
+  if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
+  const int stages = dec_attn_stages(dm, dm->K);
+  const int smem = dec::attn_smem(stages, dm->Lq, dm->K, dm->L / S, dec::max_win_slabs(dm->w)).total;
+  auto kern = dec::dec_attn_kernel<true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const float sl2 = (float)(1.0 / sqrt((double)dm->d) * 1.4426950408889634);
+  const int R = dec_attn_ranges(dm);
+  if (launch_pdl(kern, dim3(dm->B * dm->Hkv * R), dim3(dec::AT_THREADS), smem, st, kmap, vmap,
+                 static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                 static_cast<const __nv_bfloat16*>(q), q_pos, idx, dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->K, dm->w,
+                 dm->flags, R, stages, sl2, o_part, ow_part, ml_part) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const long long items = (long long)dm->B * dm->Lq * dm->Hq;
+  if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, st, q_pos, idx, z_sel,
+                 (const float*)o_part, (const float*)ow_part, (const float2*)ml_part, dm->B, dm->L, dm->Lq, dm->Hq,
+                 dm->Hkv, dm->K, dm->w, dm->flags, static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  return RDL_OK;
+}
+
+rdl_status swa_decode(const void* q, const int32_t* q_pos, const void* k, const void* v, const rdl_dims* dm, void* o,
+                      float* lse, void* workspace, cudaStream_t st) {
+  const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
+  const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
+  float* ow_part = static_cast<float*>(workspace);
+  float2* ml_part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + align256(sizeof(float) * rows * nwt * dm->d));
+  const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
+  CUtensorMap kmap, vmap;
+  if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
+  const int stages = dec_attn_stages(dm, 0);
+  const int smem = dec::attn_smem(stages, dm->Lq, 0, dm->L / S, (int)nwt).total;
+  auto kern = dec::dec_attn_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const float sl2 = (float)(1.0 / sqrt((double)dm->d) * 1.4426950408889634);
+  const int R = dec_attn_ranges(dm);
+  if (launch_pdl(kern, dim3(dm->B * dm->Hkv * R), dim3(dec::AT_THREADS), smem, st, kmap, vmap,
+                 static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                 static_cast<const __nv_bfloat16*>(q), q_pos, (const int32_t*)nullptr, dm->L, dm->Lq, dm->Hq,
+                 dm->Hkv, 0, dm->w, dm->flags, R, stages, sl2, (float*)nullptr, ow_part, ml_part) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  const long long items = (long long)dm->B * dm->Lq * dm->Hq;
+  if (launch_pdl(dec::dec_comb_kernel<false>, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, st, q_pos,
+                 (const int32_t*)nullptr, (const float*)nullptr, (const float*)nullptr, (const float*)ow_part,
+                 (const float2*)ml_part, dm->B, dm->L, dm->Lq, dm->Hq, dm->Hkv, 0, dm->w, dm->flags,
+                 static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  return RDL_OK;
 }
 
 rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const void* w_down,
@@ -349,9 +578,10 @@ const char* rdl_status_string(rdl_status s) {
 
 size_t rdl_workspace_bytes(int which, const rdl_dims* dims, rdl_dtype dtype) {
   if (!route_dims_ok(dims) || !dtype_ok(dtype)) return 0;
-  if (which == RDL_WS_SCORE) return score_ws(dims, dtype).total;
-  if (which == RDL_WS_ATTN) return attn_ws(dims, dtype).total;
-  if (which == RDL_WS_SWA) return swa_ws(dims, dtype);
+  const rdl_dims dm = clamp_w(dims);     // the calls size their workspace on the clamped radius
+  if (which == RDL_WS_SCORE) return score_ws(&dm, dtype).total;
+  if (which == RDL_WS_ATTN) return attn_ws(&dm, dtype).total;
+  if (which == RDL_WS_SWA) return swa_ws(&dm, dtype);
   return 0;
 }
 
@@ -402,6 +632,8 @@ rdl_status rdl_route_score_topk(const void* q, const int32_t* q_pos, const void*
   if (!residual) dm.r = 0;
   if (ws_bytes < score_ws(&dm, dtype).total) return RDL_ERR_WORKSPACE;
   const cudaStream_t st = as_stream(stream);
+  if (dec_score_ok(&dm, dtype))
+    return score_decode(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel, workspace, st);
   if (fast_score(&dm, dtype))
     return score_fast(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel, workspace, st);
   return dtype == RDL_BF16 ? score_impl<__nv_bfloat16>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx,
@@ -430,6 +662,8 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
   const AttnWs wl = attn_ws(dims, dtype);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RDL_ERR_INVALID_ARG;
   if (ws_bytes < wl.total) return RDL_ERR_WORKSPACE;
+  if (dec_attn_ok(dims, dtype) && dec_attn_stages(dims, dims->K) > 0)
+    return attn_decode(q, q_pos, k, v, idx, z_sel, dims, o, lse, workspace, st);
   char* ws = static_cast<char*>(workspace);
   float* o_loc = reinterpret_cast<float*>(ws + wl.o_loc);
   float* lam_loc = reinterpret_cast<float*>(ws + wl.lam_loc);
@@ -498,6 +732,11 @@ rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, cons
                              : generic_attn<float, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st);
   }
   const size_t need = swa_ws(dims, dtype);
+  if (dec_swa_ok(dims, dtype) && dec_attn_stages(dims, 0) > 0 && workspace) {
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RDL_ERR_INVALID_ARG;
+    if (ws_bytes < need) return RDL_ERR_WORKSPACE;
+    return swa_decode(q, q_pos, k, v, dims, o, lse, workspace, st);
+  }
   if (need == 0 || !workspace) return launch_window_mma<0>(q, q_pos, k, v, dims, o, lse, nullptr, nullptr, 1, st);
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RDL_ERR_INVALID_ARG;
   if (ws_bytes < need) return RDL_ERR_WORKSPACE;

@@ -1,0 +1,1122 @@
+// Route layer and sliding window for decode blocks: a few query rows (at most 64 per
+// sequence) against a long cached context.  Same definitions as the prefill kernels
+// (Prefilling-dLLM v2, Figure 3 caption; Table 3 for the window and the remote chunks),
+// organised for this shape, where the bytes that must come from HBM are the cached
+// summaries (fp32, read once) and the K/V slabs of the selected chunks:
+//
+//   dec_t_kernel      t = x W_down, one cluster of 8 CTAs: each CTA contracts one slice of
+//                     the hidden size on tensor cores, the partial products are summed in a
+//                     fixed order through distributed shared memory.
+//   dec_score_kernel  CTA = (batch, query head, chunk range).  Before its dependency wait it
+//                     starts TMA loads of its summary rows into shared memory, so the one
+//                     pass over the summaries overlaps the residual.  Then
+//                     q_res = q + t W_up for its head (tensor cores) and the split-bf16
+//                     score z = tau q_res.s - lambda H over the range.
+//   dec_topk_kernel   CTA = (batch, query row, KV group): zeta = max over the group's heads,
+//                     exact top-K (radix select), per-head scores of the selected chunks.
+//   dec_attn_kernel   chunk-major: a CTA owns one (batch, group, chunk range), finds in idx
+//                     every (row, slot) that selected a chunk of its range, streams each
+//                     selected chunk's K/V once through a TMA ring and computes the
+//                     second-level softmax output of every row that selected it; window CTAs
+//                     run the bidirectional local window of 4 rows each.
+//   dec_comb_kernel   one partition per (row, head): Z = e^lambda_loc + sum_c e^{z_c} and
+//                     o = (e^lambda_loc o_loc + sum_c e^{z_c} o_c) / Z, in a fixed order.
+//
+// The kernels of one call are chained with programmatic dependent launch: every kernel
+// waits (griddepcontrol.wait) before it touches anything an earlier kernel writes, and
+// allows its dependent to launch only after that wait, so the early start of a dependent
+// never reads data older than the call's own inputs.
+#pragma once
+#include <cooperative_groups.h>
+#include "common.cuh"
+#include "tc.cuh"
+#include "score.cuh"
+
+// Phase markers: empty unless a build defines them (kernel id, slot).
+#ifndef RDL_TRACE_POINT
+#define RDL_TRACE_POINT(kernel, slot)
+#endif
+
+namespace rdl {
+namespace dec {
+
+namespace cg = cooperative_groups;
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// fp32 pair -> (hi, lo) packed bf16 pairs with x = hi + lo to ~2^-17 relative.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+  const __nv_bfloat162 hh = __halves2bfloat162(h0, h1);
+  const __nv_bfloat162 ll = __floats2bfloat162_rn(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+  hi = *reinterpret_cast<const uint32_t*>(&hh);
+  lo = *reinterpret_cast<const uint32_t*>(&ll);
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// =====================================================================================
+// dec_t_kernel: t[M, r] = x[M, D] W_down[D, r] (bf16 inputs, exact products, fp32 sums).
+// One cluster of 8 CTAs; CTA `rank` owns hidden slice [rank*slice, rank*slice + slice).
+// =====================================================================================
+constexpr int TK_CL = 8;
+constexpr int TK_KMAX = 512;                                // hidden columns per load batch
+
+// shared memory of dec_t_kernel for `rows` (multiple of 16) query rows, rank r and a batch
+// of kc hidden columns (multiple of 64): per 64-column block, x [rows][128 B] and
+// W_down [64][128 B] per 64 columns of r (TMA boxes, 128-byte swizzle); partial t [rows][r].
+__host__ __device__ inline int tk_smem(int rows, int r, int kc) {
+  return 1024 + (kc / 64) * (rows * 128 + (r / 64) * 8192) + rows * r * 4 + 16;
+}
+
+__global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
+    dec_t_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, int M,
+                 int D, int r, int kc, float* __restrict__ t) {
+  extern __shared__ unsigned char tk_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(tk_raw) + 1023) & ~uintptr_t(1023));
+  RDL_TRACE_POINT(0, 0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Mt = (M + 15) >> 4, rows = Mt * 16;
+  const int nkb = kc / 64, nnb = r / 64;
+  const int xblk = rows * 128, wblk = nnb * 8192;
+  unsigned char* xs = base;                                    // [nkb][rows][128 B]
+  unsigned char* ws = xs + nkb * xblk;                         // [nkb][nnb][64][128 B]
+  float* part = reinterpret_cast<float*>(ws + nkb * wblk);     // [rows][r]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(part + rows * r);
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
+  RDL_TRACE_POINT(0, 1);
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int slice = ((D + TK_CL * 64 - 1) / (TK_CL * 64)) * 64;
+  const int k0 = min(D, rank * slice), k1 = min(D, k0 + slice);
+  const int npairs = r / 16, ntask = Mt * npairs;
+  float acc[4][2][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int n = 0; n < 2; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
+
+  unsigned phase = 0;
+  for (int kb = k0; kb < k1; kb += kc) {
+    const int nb = min(kc, k1 - kb) / 64;                      // 64-column blocks in this batch
+    if (tid == 0) {
+      tc::mbar_arrive_expect_tx(bar, (unsigned)(nb * (xblk + wblk)));
+      for (int j = 0; j < nb; ++j) {
+        tc::tma_load_2d(xs + j * xblk, &xmap, kb + 64 * j, 0, bar);
+        for (int n = 0; n < nnb; ++n) tc::tma_load_2d(ws + j * wblk + n * 8192, &wmap, 64 * n, kb + 64 * j, bar);
+      }
+    }
+    if (!tc::mbar_wait(bar, phase)) break;
+    phase ^= 1u;
+    RDL_TRACE_POINT(0, 2);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int task = warp + 8 * a;
+      if (task >= ntask) break;
+      const int mt = task / npairs, np = task % npairs;
+      for (int ks = 0; ks < nb * 4; ++ks) {
+        const unsigned char* xb = xs + (ks >> 2) * xblk;
+        const unsigned char* wb = ws + (ks >> 2) * wblk + (np >> 2) * 8192;
+        const int kq = (ks & 3) * 16;
+        uint32_t af[4];
+        const int ra = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        ldsm_x4(smem_u32(xb + tc::sw128(ra, kq + 8 * (lane >> 4))), af[0], af[1], af[2], af[3]);
+        uint32_t b0, b1, b2, b3;
+        const int mi = lane >> 3, kk = kq + 8 * (mi & 1) + (lane & 7), nn = ((2 * np) & 7) * 8 + 8 * (mi >> 1);
+        ldsm_x4_t(smem_u32(wb + tc::sw128(kk, nn)), b0, b1, b2, b3);
+        mma_bf16(acc[a][0], af, b0, b1);
+        mma_bf16(acc[a][1], af, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  RDL_TRACE_POINT(0, 3);
+  // push reduction: CTA `rank` stores its partial of row block j straight into CTA j's
+  // shared memory (recv[rank]); one cluster barrier, then every CTA sums its own block in
+  // rank order, so the result is the same on every run
+  const int gq = lane >> 2, tq = lane & 3;
+  const int rows_per = (M + TK_CL - 1) / TK_CL;
+  float* recv = part;                                          // [TK_CL][rows_per][r]
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int task = warp + 8 * a;
+    if (task >= ntask) break;
+    const int mt = task / npairs, np = task % npairs;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = mt * 16 + gq + 8 * hr;
+      if (row >= M) continue;
+      const int owner = row / rows_per, lr = row - owner * rows_per;
+      float* dst = cl.map_shared_rank(recv, owner) + ((size_t)rank * rows_per + lr) * r;
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int col = (2 * np + n) * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(dst + col) = make_float2(acc[a][n][2 * hr], acc[a][n][2 * hr + 1]);
+      }
+    }
+  }
+  cl.sync();
+  const int r0 = rank * rows_per, nr = max(0, min(rows_per, M - r0));
+  for (int e = tid; e < nr * r; e += 256) {
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < TK_CL; ++c) sum += recv[(size_t)c * rows_per * r + e];
+    t[(size_t)r0 * r + e] = sum;
+  }
+  RDL_TRACE_POINT(0, 4);
+}
+
+// =====================================================================================
+// dec_score_kernel: CTA = (chunk range, query head h, batch b); 8 warps.
+// MT = m-tiles of 16 query rows (rows = Lq <= 16*MT).
+// Shared memory:
+//   ring   nstg stages of boxr summary rows, each [4 slices][boxr][32 fp32] with the
+//          128-byte swizzle of the TMA box (16-byte unit ^ row % 8)
+//   wup    W_up columns of head h: [r][128] bf16, unit-swizzled (ldmatrix.trans)
+//   qh     q rows of head h: [16*MT][136] bf16 (padded rows)
+//   qt     q_res rows: [16*MT][132] fp32 (padded rows)
+// =====================================================================================
+struct ScoreSmem {
+  int ring, wup, qh, qt, ts, hs, ps, bar, total;
+};
+__host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nstg, int ncr) {
+  ScoreSmem s{};
+  int off = 0;
+  s.ring = off; off += nstg * boxr * 512;
+  s.wup = off;  off += (r > 0 ? r : 1) * 256;
+  s.qh = off;   off += MT * 16 * 272;
+  s.qt = off;   off += MT * 16 * 528;
+  s.ts = off;   off += MT * 16 * (r + 8) * 4;
+  s.hs = off;   off += ((ncr + 3) / 4) * 16;
+  s.ps = off;   off += 64 * 4;
+  s.bar = off;  off += 8 * nstg;
+  s.total = off + 1024;       // slack for aligning the base to 1024 bytes
+  return s;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(256, 1)
+    dec_score_kernel(const __grid_constant__ CUtensorMap smap, const float* __restrict__ smap_base,
+                     const __nv_bfloat16* __restrict__ q,
+                     const int32_t* __restrict__ q_pos, const float* __restrict__ t,
+                     const __nv_bfloat16* __restrict__ w_up, const float* __restrict__ entropy, int Lq, int L,
+                     int Hq, int r, int w, float tau, float lambda, int ncr, int boxr, int nbox, int nstg,
+                     float* __restrict__ z_all) {
+  constexpr int D = 128;
+  constexpr int NG = 8 / MT;                  // warps per m-tile (n-groups)
+  extern __shared__ unsigned char sc_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sc_raw) + 1023) & ~uintptr_t(1023));
+  const ScoreSmem L_ = score_smem(MT, r, boxr, nstg, ncr);
+  unsigned char* ring = base + L_.ring;
+  unsigned char* wup = base + L_.wup;
+  unsigned char* qh = base + L_.qh;
+  float* qt = reinterpret_cast<float*>(base + L_.qt);
+  float* ts = reinterpret_cast<float*>(base + L_.ts);
+  float* hs = reinterpret_cast<float*>(base + L_.hs);
+  int* ps = reinterpret_cast<int*>(base + L_.ps);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + L_.bar);
+
+  const int C = L / S;
+  const int b = blockIdx.z, h = blockIdx.y;
+  RDL_TRACE_POINT(1, 0);
+  const int c0 = blockIdx.x * ncr, c1 = min(C, c0 + ncr);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int mw = warp % MT, ng = warp / MT;
+  if (c0 >= C) {
+    grid_dep_wait();
+    return;
+  }
+  const int nb = min(nbox, (c1 - c0 + boxr - 1) / boxr);
+  const size_t srow0 = (size_t)(b * Hq + h) * C + c0;
+  // ---- prologue: only TMA and cp.async.cg loads of inputs (no kernel of this call writes
+  // them, and this kernel is launched early only behind dec_t_kernel, which has waited)
+  if (tid == 0) {
+    for (int s = 0; s < nstg; ++s) tc::mbar_init(&full[s], 1);
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int bx = 0; bx < nb && bx < nstg; ++bx) {
+      tc::mbar_arrive_expect_tx(&full[bx], (unsigned)boxr * 512u);
+      tc::tma_load_3d(ring + bx * boxr * 512, &smap, 0, (int)(srow0 + (size_t)bx * boxr), 0, &full[bx]);
+    }
+  }
+  for (int e = tid; e < r * 16; e += 256) {
+    const int kk = e >> 4, u = e & 15;
+    cp_async16(smem_u32(wup + kk * 256 + ((u ^ (kk & 7)) << 4)), w_up + (size_t)kk * Hq * D + h * D + u * 8);
+  }
+  for (int e = tid; e < Lq * 16; e += 256) {
+    const int i = e >> 4, u = e & 15;
+    cp_async16(smem_u32(qh + i * 272 + u * 16), q + ((size_t)(b * Lq + i) * Hq + h) * D + u * 8);
+  }
+  cp_async_commit();
+  for (int j = tid; j < c1 - c0; j += 256) hs[j] = __ldcg(entropy + (size_t)(b * Hq + h) * C + c0 + j);
+  if (tid < MT * 16) ps[tid] = tid < Lq ? (q_pos ? __ldcg(q_pos + (size_t)b * Lq + tid) : tid) : INT_MIN;
+  // rows beyond the ring: pulled into L2 now, loaded into the ring when a stage frees
+  for (int bx = nstg + (tid >> 5); bx < nb; bx += 8) {
+    const char* src = reinterpret_cast<const char*>(smap_base) + (srow0 + (size_t)bx * boxr) * 512;
+    const int bytes = min(boxr, (c1 - c0) - bx * boxr) * 512;
+    for (int off = (tid & 31) * 4096; off < bytes; off += 32 * 4096)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src + off), "r"(min(4096, bytes - off))
+                   : "memory");
+  }
+
+  grid_dep_wait();      // t is written by dec_t_kernel
+  grid_dep_launch();
+  RDL_TRACE_POINT(1, 1);
+  if (r > 0) {
+    const int nu = r / 4;                       // 16-byte units per t row
+    for (int e = tid; e < Lq * nu; e += 256) {
+      const int i = e / nu, u = e % nu;
+      cp_async16(smem_u32(ts + i * (r + 8) + u * 4), t + (size_t)(b * Lq + i) * r + u * 4);
+    }
+  }
+  cp_async_commit();
+
+  // ---- q_res = q + t W_up for this warp's m-tile and n-group (tensor cores, t split)
+  {
+    constexpr int NPW = 16 / NG;              // n-tiles (of 8 columns) per warp
+    float ua[NPW][4];
+#pragma unroll
+    for (int n = 0; n < NPW; ++n) ua[n][0] = ua[n][1] = ua[n][2] = ua[n][3] = 0.f;
+    const int row0 = mw * 16 + gq, row1 = row0 + 8;
+    cp_async_wait<0>();
+    __syncthreads();
+    RDL_TRACE_POINT(1, 2);
+    for (int kk = 0; kk < r / 16; ++kk) {
+      uint32_t ahi[4], alo[4];
+      {
+        const int ca = 16 * kk + 2 * tq, rs = r + 8;
+        const float2 z2 = make_float2(0.f, 0.f);
+        const float2 v0 = row0 < Lq ? *reinterpret_cast<const float2*>(ts + row0 * rs + ca) : z2;
+        const float2 v1 = row1 < Lq ? *reinterpret_cast<const float2*>(ts + row1 * rs + ca) : z2;
+        const float2 v2 = row0 < Lq ? *reinterpret_cast<const float2*>(ts + row0 * rs + ca + 8) : z2;
+        const float2 v3 = row1 < Lq ? *reinterpret_cast<const float2*>(ts + row1 * rs + ca + 8) : z2;
+        split2(v0.x, v0.y, ahi[0], alo[0]);
+        split2(v1.x, v1.y, ahi[1], alo[1]);
+        split2(v2.x, v2.y, ahi[2], alo[2]);
+        split2(v3.x, v3.y, ahi[3], alo[3]);
+      }
+#pragma unroll
+      for (int n = 0; n < NPW; n += 2) {
+        const int nt = ng * NPW + n;
+        uint32_t b0, b1, b2, b3;
+        const int mi = lane >> 3, k = 16 * kk + 8 * (mi & 1) + (lane & 7), un = nt + (mi >> 1);
+        ldsm_x4_t(smem_u32(wup + k * 256 + ((un ^ (k & 7)) << 4)), b0, b1, b2, b3);
+        mma_bf16(ua[n], ahi, b0, b1);
+        mma_bf16(ua[n], alo, b0, b1);
+        mma_bf16(ua[n + 1], ahi, b2, b3);
+        mma_bf16(ua[n + 1], alo, b2, b3);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NPW; ++n) {
+      const int col = (ng * NPW + n) * 8 + 2 * tq;
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = mw * 16 + gq + 8 * hr;
+        const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162*>(qh + row * 272 + col * 2);
+        const float2 qf = __bfloat1622float2(qv);
+        qt[row * 132 + col] = qf.x + ua[n][2 * hr];
+        qt[row * 132 + col + 1] = qf.y + ua[n][2 * hr + 1];
+      }
+    }
+  }
+  __syncthreads();
+  // ---- A fragments of q_res (hi/lo) for this warp's m-tile, all 8 k-steps
+  uint32_t ahi[8][4], alo[8][4];
+  {
+    const int row0 = mw * 16 + gq, row1 = row0 + 8;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int ca = 16 * ks + 2 * tq;
+      const float2 v0 = *reinterpret_cast<const float2*>(qt + row0 * 132 + ca);
+      const float2 v1 = *reinterpret_cast<const float2*>(qt + row1 * 132 + ca);
+      const float2 v2 = *reinterpret_cast<const float2*>(qt + row0 * 132 + ca + 8);
+      const float2 v3 = *reinterpret_cast<const float2*>(qt + row1 * 132 + ca + 8);
+      split2(v0.x, v0.y, ahi[ks][0], alo[ks][0]);
+      split2(v1.x, v1.y, ahi[ks][1], alo[ks][1]);
+      split2(v2.x, v2.y, ahi[ks][2], alo[ks][2]);
+      split2(v3.x, v3.y, ahi[ks][3], alo[ks][3]);
+    }
+  }
+  const int prow[2] = {ps[mw * 16 + gq], ps[mw * 16 + gq + 8]};
+  RDL_TRACE_POINT(1, 3);
+  const int irow[2] = {mw * 16 + gq, mw * 16 + gq + 8};
+  // ---- scores over the range, box by box as the TMA loads land.  Each landed box is first
+  // rewritten in place: every 128-byte segment (32 fp32 of one summary row) becomes 32 bf16
+  // hi terms (logical 16-byte units 0-3) and 32 bf16 lo terms (units 4-7), x = hi + lo to
+  // ~2^-17, keeping the unit ^ (row % 8) swizzle so the fragment loads stay conflict-free.
+  const int ntb = boxr / 8;
+  for (int bx = 0; bx < nb; ++bx) {
+    const int s = bx % nstg;
+    if (!tc::mbar_wait(&full[s], (unsigned)(bx / nstg) & 1u)) break;
+    if (bx == 0) RDL_TRACE_POINT(1, 4);
+    unsigned char* stg = ring + s * boxr * 512;
+    for (int seg = tid; seg < 4 * boxr; seg += 256) {
+      const int rr = seg % boxr;
+      unsigned char* sp = stg + (seg / boxr) * boxr * 128 + rr * 128;
+      const int sw = rr & 7;
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const float4*>(sp + ((u ^ sw) << 4));
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        split2(v[u].x, v[u].y, hi[2 * u], lo[2 * u]);
+        split2(v[u].z, v[u].w, hi[2 * u + 1], lo[2 * u + 1]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        *reinterpret_cast<uint4*>(sp + ((u ^ sw) << 4)) = make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+        *reinterpret_cast<uint4*>(sp + (((4 + u) ^ sw) << 4)) =
+            make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
+      }
+    }
+    __syncthreads();
+    const uint32_t st = smem_u32(stg);
+    const int cb = c0 + bx * boxr;
+    for (int nt = ng; nt < ntb; nt += NG) {
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+      const int rl = nt * 8 + (lane & 7), mj = lane >> 3;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        // matrices: hi dims d0..+7, hi d0+8..+15, lo d0..+7, lo d0+8..+15 of chunk rows nt*8..+7
+        const int un = (mj >= 2 ? 4 : 0) + ((16 * ks) & 31) / 8 + (mj & 1);
+        uint32_t bh0, bh1, bl0, bl1;
+        ldsm_x4(st + (ks >> 1) * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
+        mma_bf16(a0, ahi[ks], bh0, bh1);
+        mma_bf16(a1, ahi[ks], bl0, bl1);
+        mma_bf16(a2, alo[ks], bh0, bh1);
+      }
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int i = irow[hr];
+        if (i >= Lq) continue;
+        const int cc = cb + nt * 8 + 2 * tq;
+        float z[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = cc + e;
+          const float acc = a0[2 * hr + e] + (a1[2 * hr + e] + a2[2 * hr + e]);
+          z[e] = (c < c1 && chunk_eligible(c, prow[hr], w)) ? tau * acc - lambda * hs[c - c0] : -INFINITY;
+        }
+        float* zr = z_all + ((size_t)(b * Hq + h) * Lq + i) * C;
+        if (cc + 1 < c1 && ((C & 1) == 0)) {
+          *reinterpret_cast<float2*>(zr + cc) = make_float2(z[0], z[1]);
+        } else {
+          if (cc < c1) zr[cc] = z[0];
+          if (cc + 1 < c1) zr[cc + 1] = z[1];
+        }
+      }
+    }
+    __syncthreads();                       // stage s consumed by every warp
+    if (tid == 0 && bx + nstg < nb) {
+      tc::fence_proxy_async();
+      tc::mbar_arrive_expect_tx(&full[s], (unsigned)boxr * 512u);
+      tc::tma_load_3d(ring + s * boxr * 512, &smap, 0, (int)(srow0 + (size_t)(bx + nstg) * boxr), 0, &full[s]);
+    }
+  }
+  RDL_TRACE_POINT(1, 5);
+}
+
+// =====================================================================================
+// dec_topk_kernel: CTA = (query row i, group g, batch b), 256 threads.  The G score rows
+// of (i, g) arrive in shared memory in one cp.async batch when C % 4 == 0 and G*C fits
+// (ZS = true); otherwise they are read from global memory.
+// =====================================================================================
+constexpr int DK_MAXZ = 8 * 4096;           // floats of staged score rows
+
+// Top-K of the group max by a candidate filter.  Keys are (order_key(zeta), ~chunk) packed
+// in 64 bits, so larger means better with ties to the smaller chunk.  Every warp finds its
+// q-th largest key (q = ceil(K / 8)); the smallest of those eight bounds the K-th largest key
+// from below (each warp holds q keys at or above its own bound), so every key of the top K is
+// among the candidates at or above it.  The candidates (typically a few more than K) are
+// ranked exactly; more than DK_MAXCAND of them (heavy ties) falls back to the radix select.
+constexpr int DK_MAXCAND = 256;
+
+template <bool ZS, int MAXM>
+__global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__ z_all,
+                                                       const int32_t* __restrict__ q_pos, int Lq, int L,
+                                                       int Hq, int Hkv, int K, int32_t* __restrict__ idx,
+                                                       float* __restrict__ z_sel) {
+  extern __shared__ __align__(128) uint32_t dk_smem[];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned whist[8][256];
+  __shared__ int warp_sums[8];
+  __shared__ int sel_s[64];
+  __shared__ int bc[3];
+  __shared__ unsigned long long wbound[8];
+  __shared__ unsigned long long cand[DK_MAXCAND];
+  __shared__ int ncand_s;
+  __shared__ __align__(8) uint64_t zbar;
+  RDL_TRACE_POINT(2, 0);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&zbar, 1);
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
+  RDL_TRACE_POINT(2, 1);
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  uint32_t* keys = dk_smem;                                        // [C]
+  float* zs = reinterpret_cast<float*>(dk_smem + ((C + 3) & ~3));  // [G][C] (ZS)
+  const float* z0 = z_all + ((size_t)(b * Hq + g * G) * Lq + i) * C;
+  const size_t hstride = (size_t)Lq * C;
+  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+  int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
+  if (is_mask_slot(p)) {
+    for (int e = tid; e < K * G; e += 256) {
+      const int k = e % K, hl = e / K;
+      if (hl == 0) irow[k] = -1;
+      z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
+    }
+    return;
+  }
+  if (ZS) {
+    // the group's G score rows: G bulk copies on one barrier
+    if (tid == 0) {
+      tc::mbar_arrive_expect_tx(&zbar, (unsigned)(G * C * 4));
+      for (int hl = 0; hl < G; ++hl) tc::bulk_load(zs + hl * C, z0 + hl * hstride, (unsigned)(C * 4), &zbar);
+    }
+    (void)tc::mbar_wait(&zbar, 0);
+  }
+  const uint32_t kneg = order_key(-INFINITY);
+  // thread t owns chunks t + 256 m (m < MAXM, C <= 256 MAXM); packed keys stay in registers
+  const int nm = (C + 255) / 256;
+  unsigned long long pk[MAXM];
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    pk[m] = 0ull;
+    const int c = tid + 256 * m;
+    if (m < nm && c < C) {
+      float zz;
+      if (ZS) {
+        zz = zs[c];
+        for (int hl = 1; hl < G; ++hl) zz = fmaxf(zz, zs[hl * C + c]);
+      } else {
+        zz = z0[c];
+        for (int hl = 1; hl < G; ++hl) zz = fmaxf(zz, z0[hl * hstride + c]);
+      }
+      const uint32_t key = order_key(zz);
+      keys[c] = key;
+      if (key > kneg) pk[m] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)c);
+    }
+  }
+  RDL_TRACE_POINT(2, 2);
+  // per-warp q-th largest packed key (0 when the warp has fewer than q valid keys)
+  const int qk = (K + 7) / 8;
+  {
+    unsigned long long last = ~0ull, bound = 0ull;
+    for (int r = 0; r < qk; ++r) {
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m)
+        if (pk[m] < last && pk[m] > best) best = pk[m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long x = __shfl_xor_sync(0xffffffffu, best, o);
+        best = x > best ? x : best;
+      }
+      last = best;
+      bound = best;
+      if (best == 0ull) break;
+    }
+    if (lane == 0) wbound[warp] = bound;
+  }
+  if (tid == 0) ncand_s = 0;
+  __syncthreads();
+  unsigned long long L0 = wbound[0];
+#pragma unroll
+  for (int w8 = 1; w8 < 8; ++w8) L0 = wbound[w8] < L0 ? wbound[w8] : L0;
+  if (L0 == 0ull) L0 = 1ull;      // fewer than K valid keys in some warp: every valid key is a candidate
+  // candidates: keys >= L0
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    if (pk[m] >= L0) {
+      const int slot = atomicAdd(&ncand_s, 1);
+      if (slot < DK_MAXCAND) cand[slot] = pk[m];
+    }
+  }
+  __syncthreads();
+  const int ncand = ncand_s;
+  int nsel;
+  if (ncand <= DK_MAXCAND) {
+    // exact rank of each candidate (keys are distinct)
+    if (tid < ncand) {
+      const unsigned long long mine = cand[tid];
+      int rank = 0;
+      for (int e = 0; e < ncand; ++e) rank += cand[e] > mine;
+      if (rank < K) sel_s[rank] = (int)(0xffffffffu - (uint32_t)(mine & 0xffffffffull));
+    }
+    nsel = min(ncand, K);
+    __syncthreads();
+    // ascending chunk order
+    int c_mine = 0, pos = 0;
+    if (tid < nsel) {
+      c_mine = sel_s[tid];
+      for (int e = 0; e < nsel; ++e) pos += sel_s[e] < c_mine;
+    }
+    __syncthreads();
+    if (tid < nsel) sel_s[pos] = c_mine;
+    __syncthreads();
+  } else {
+    __syncthreads();
+    nsel = cta_select_topk(keys, C, K, hist, whist, warp_sums, bc, sel_s);
+  }
+  RDL_TRACE_POINT(2, 3);
+  for (int e = tid; e < K * G; e += 256) {
+    const int k = e % K, hl = e / K;
+    const int c = k < nsel ? sel_s[k] : -1;
+    if (hl == 0) irow[k] = c;
+    float z = -INFINITY;
+    if (c >= 0) z = ZS ? zs[hl * C + c] : z0[hl * hstride + c];
+    z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = z;
+  }
+  RDL_TRACE_POINT(2, 4);
+}
+
+// =====================================================================================
+// dec_attn_kernel: chunk-major two-level attention for decode blocks.
+//
+// Work items: for KV group (b, g), every 64-key slab c that some row needs -- because the
+// row selected chunk c (a chunk task: second-level softmax over the 63 content keys) or
+// because slab c overlaps the row's window (a window task: the window keys of that slab).
+// The R CTAs of a group all build the same histogram of tasks per slab from idx and the
+// row positions and split the prefix of (row pairs + one slab load) into R equal shares,
+// so a chunk that every row selected costs one CTA as much as many sparse ones.  A CTA
+// streams its slabs once through a TMA ring; each consumer warp computes two tasks of a
+// slab at once (M = 16 = two rows x 8 head slots) with the probabilities kept in
+// registers (no shared-memory round trip), and writes one partial per task:
+//   chunk task  -> o_part[b,i,g,k]  = softmax-normalised output of chunk idx[k]
+//   window task -> ow_part[b,i,g,s] = unnormalised sum, ml_part = (max, sum) of slab s
+// dec_comb_kernel merges the partials of a row in a fixed order.
+// =====================================================================================
+constexpr int AT_CONS = 15;
+constexpr int AT_THREADS = (AT_CONS + 1) * 32;
+constexpr int AT_STAGE_BYTES = 32768;
+constexpr int AT_MAXC = 2048;            // chunks per sequence on this path
+constexpr int AT_QROWS = 32;             // query rows per sequence on this path
+
+// window slabs a row at position p touches: [wlo(p), whi(p)] (w >= 0)
+__device__ __forceinline__ int win_lo(int p, int w) { return max(0, p - w) / S; }
+__device__ __forceinline__ int win_hi(int p, int w, int L) { return min(L - 1, p + w) / S; }
+// most window slabs of one row: 2w+1 keys span at most 2w/64 + 2 slabs
+__host__ __device__ inline int max_win_slabs(int w) { return w < 0 ? 0 : (2 * w) / S + 2; }
+
+struct AttnSmem {
+  int ring, qs, idx, pos, hist, pre, list, bar, misc, total;
+};
+__host__ __device__ inline AttnSmem attn_smem(int stages, int Lq, int K, int C, int nwt) {
+  AttnSmem s{};
+  int off = 0;
+  s.ring = off; off += stages * AT_STAGE_BYTES;
+  s.qs = off;   off += Lq * 2048;
+  s.idx = off;  off += ((Lq * K + 3) & ~3) * 4;
+  s.pos = off;  off += ((Lq + 3) & ~3) * 4;
+  s.hist = off; off += ((C + 3) & ~3) * 4;
+  s.pre = off;  off += ((C + 3) & ~3) * 4;
+  s.list = off; off += ((Lq * (K + nwt) + 3) & ~3) * 4;
+  s.bar = off;  off += 16 * stages;
+  s.misc = off; off += 256;
+  s.total = off + 1024;
+  return s;
+}
+
+// byte offset of (row, col) in a K/V slab tile ([2 halves][64 rows][128 B], 128-byte swizzle)
+__device__ __forceinline__ uint32_t kv_off(int row, int col) {
+  return (uint32_t)((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
+}
+
+// Exclusive scan of one int per thread over the whole CTA (blockDim.x <= 1024); returns the
+// thread's exclusive prefix and the CTA total.  ws: blockDim.x / 32 ints of shared memory.
+__device__ __forceinline__ int cta_excl_scan(int v, int* ws, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) ws[warp] = x;
+  __syncthreads();
+  int basev = 0, tot = 0;
+  for (int w8 = 0; w8 < nw; ++w8) {
+    const int t = ws[w8];
+    if (w8 < warp) basev += t;
+    tot += t;
+  }
+  __syncthreads();
+  total = tot;
+  return basev + x - v;
+}
+
+// task word: row (6 bits) << 8 | kind (window = 128) | slot (7 bits)
+constexpr int TASK_WIN = 128;
+
+template <bool ROUTE>
+__global__ void __launch_bounds__(AT_THREADS, 1)
+    dec_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const __nv_bfloat16* __restrict__ kv_base_k, const __nv_bfloat16* __restrict__ kv_base_v,
+                    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
+                    const int32_t* __restrict__ idx, int L, int Lq, int Hq, int Hkv, int K, int w, int flags,
+                    int R, int stages, float sl2, float* __restrict__ o_part, float* __restrict__ ow_part,
+                    float2* __restrict__ ml_part) {
+  constexpr int D = 128;
+  extern __shared__ unsigned char at_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(at_raw) + 1023) & ~uintptr_t(1023));
+  const int C = L / S, G = Hq / Hkv;
+  const int nwt = max_win_slabs(w);
+  const int Kt = ROUTE ? K : 0;
+  const AttnSmem SL = attn_smem(stages, Lq, Kt, C, nwt);
+  unsigned char* ring = base + SL.ring;
+  unsigned char* qs = base + SL.qs;
+  int* idx_s = reinterpret_cast<int*>(base + SL.idx);
+  int* pos_s = reinterpret_cast<int*>(base + SL.pos);
+  int* hist = reinterpret_cast<int*>(base + SL.hist);
+  int* pre = reinterpret_cast<int*>(base + SL.pre);
+  int* list = reinterpret_cast<int*>(base + SL.list);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + SL.bar);
+  uint64_t* empty = full + stages;
+  int* misc = reinterpret_cast<int*>(base + SL.misc);   // [0] c_lo [1] c_hi [2] abort [3..4] scan
+  RDL_TRACE_POINT(3, 0);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int item = blockIdx.x, j = item % R, g = (item / R) % Hkv, b = item / (R * Hkv);
+  const size_t kvrow0 = (size_t)(b * Hkv + g) * L;
+
+  if (tid == 0) {
+    for (int st = 0; st < stages; ++st) {
+      tc::mbar_init(&full[st], 1);
+      tc::mbar_init(&empty[st], AT_CONS);
+    }
+    tc::mbar_fence_init();
+    misc[0] = INT_MAX;
+    misc[1] = -1;
+    misc[2] = 0;
+  }
+  grid_dep_wait();
+  grid_dep_launch();
+  RDL_TRACE_POINT(3, 1);
+
+  // ---------------- one load batch: idx rows of the group, positions, query rows
+  const int nent = Lq * Kt;
+  const int32_t* ib = ROUTE ? idx + (size_t)(b * Hkv + g) * Lq * K : nullptr;
+  if (ROUTE) {
+    if ((nent & 3) == 0) {
+      for (int e = tid; e < nent / 4; e += AT_THREADS) cp_async16(smem_u32(idx_s + 4 * e), ib + 4 * e);
+    } else {
+      for (int e = tid; e < nent; e += AT_THREADS) idx_s[e] = ib[e];
+    }
+  }
+  for (int e = tid; e < Lq; e += AT_THREADS) pos_s[e] = q_pos ? q_pos[(size_t)b * Lq + e] : e;
+  for (int e = tid; e < Lq * 8 * 16; e += AT_THREADS) {
+    const int i = e >> 7, hd = (e >> 4) & 7, u = e & 15;
+    unsigned char* dst = qs + i * 2048 + hd * 256 + ((u ^ hd) << 4);
+    if (hd < G)
+      cp_async16(smem_u32(dst), q + ((size_t)(b * Lq + i) * Hq + g * G + hd) * D + u * 8);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
+  for (int c = tid; c < C; c += AT_THREADS) hist[c] = 0;
+  cp_async_wait<0>();
+  __syncthreads();
+  RDL_TRACE_POINT(3, 4);
+  // ---------------- tasks per slab (the same on every CTA of the group)
+  auto chunk_ok = [&](int e, int c) -> bool {   // entry e of idx_s holds chunk c >= 0
+    if (c >= C) return false;
+    if (flags & RDL_FLAG_CHECKS) return chunk_eligible(c, pos_s[e / K], w);
+    return true;
+  };
+  if (ROUTE) {
+    for (int e = tid; e < nent; e += AT_THREADS) {
+      const int c = idx_s[e];
+      if (c < 0) continue;
+      if (!chunk_ok(e, c)) {
+        if (flags & RDL_FLAG_CHECKS) record_status(RDL_ERR_DEVICE_CHECK);
+        continue;
+      }
+      atomicAdd(&hist[c], 1);
+    }
+  }
+  if (w >= 0) {
+    for (int i = warp; i < Lq; i += AT_CONS + 1) {
+      const int p = pos_s[i];
+      if (ROUTE && is_mask_slot(p)) continue;
+      const int lo = win_lo(p, w), hi = win_hi(p, w, L);
+      for (int t = lo + lane; t <= hi; t += 32) atomicAdd(&hist[t], 1);
+    }
+  }
+  __syncthreads();
+  // work of slab c: its row pairs plus one slab load; exclusive prefix in chunk order.
+  // Slab c belongs to CTA floor(prefix(c) * R / total): contiguous slab ranges of equal work.
+  int* scan_ws = misc + 32;                                  // 9 ints
+  const int seg = (C + AT_THREADS - 1) / AT_THREADS;
+  const int s0 = min(C, tid * seg), s1 = min(C, s0 + seg);
+  {
+    int local = 0;
+    for (int c = s0; c < s1; ++c) {
+      const int n = hist[c];
+      local += n > 0 ? (n + 1) / 2 + 1 : 0;
+    }
+    int total;
+    int run = cta_excl_scan(local, scan_ws, total);
+    const long long W = total;
+    for (int c = s0; c < s1; ++c) {
+      const int n = hist[c];
+      if (n > 0) {
+        const int owner = (int)(((long long)run * R) / W);
+        if (owner == j) {
+          atomicMin(&misc[0], c);
+          atomicMax(&misc[1], c);
+        }
+        run += (n + 1) / 2 + 1;
+      }
+    }
+  }
+  RDL_TRACE_POINT(3, 6);
+  // task cursors: pre[c] = first list position of slab c (prefix of the task counts)
+  {
+    int local = 0;
+    for (int c = s0; c < s1; ++c) local += hist[c];
+    int total;
+    int run = cta_excl_scan(local, scan_ws, total);
+    for (int c = s0; c < s1; ++c) {
+      pre[c] = run;
+      run += hist[c];
+    }
+  }
+  __syncthreads();
+  const int c_lo = misc[0], c_hi = misc[1] + 1;     // empty when c_lo > c_hi - 1
+  const int lbase = c_lo < c_hi ? pre[c_lo] : 0;   // list positions relative to this CTA
+  const int lcap = Lq * (Kt + nwt);
+  __syncthreads();
+  if (ROUTE && c_lo < c_hi) {
+    for (int e = tid; e < nent; e += AT_THREADS) {
+      const int c = idx_s[e];
+      if (c < c_lo || c >= c_hi || !chunk_ok(e, c)) continue;
+      const int slot = atomicAdd(&pre[c], 1) - lbase;
+      if (slot < lcap) list[slot] = ((e / K) << 8) | (e % K);
+      else record_status(RDL_ERR_DEVICE_CHECK);
+    }
+  }
+  if (w >= 0 && c_lo < c_hi) {
+    for (int i = warp; i < Lq; i += AT_CONS + 1) {
+      const int p = pos_s[i];
+      if (ROUTE && is_mask_slot(p)) continue;
+      const int lo = win_lo(p, w), hi = min(win_hi(p, w, L), c_hi - 1);
+      for (int t = max(lo, c_lo) + lane; t <= hi; t += 32) {
+        const int slot = atomicAdd(&pre[t], 1) - lbase;
+        if (slot < lcap) list[slot] = (i << 8) | TASK_WIN | (t - lo);
+        else record_status(RDL_ERR_DEVICE_CHECK);
+      }
+    }
+  }
+  __syncthreads();
+  RDL_TRACE_POINT(3, 2);
+  // after the scatter pre[c] = end of slab c's tasks (absolute); start = end - hist[c]
+
+  if (warp == AT_CONS) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int u = 0;
+      int last_issued[4] = {-1, -1, -1, -1};
+      for (int c = c_lo; c < c_hi; ++c) {
+        if (hist[c] == 0) continue;
+        const int st = u % stages, n = u / stages;
+        if (n > 0 && !tc::mbar_wait(&empty[st], (unsigned)(n - 1) & 1u)) {
+          misc[2] = 1;
+          break;
+        }
+        if (misc[2]) break;
+        unsigned char* dst = ring + st * AT_STAGE_BYTES;
+        tc::mbar_arrive_expect_tx(&full[st], AT_STAGE_BYTES);
+        tc::tma_load_3d(dst, &kmap, 0, (int)(kvrow0 + (size_t)S * c), 0, &full[st]);
+        tc::tma_load_3d(dst + 16384, &vmap, 0, (int)(kvrow0 + (size_t)S * c), 0, &full[st]);
+        last_issued[st] = u;
+        ++u;
+      }
+      for (int st = 0; st < stages; ++st)
+        if (last_issued[st] >= 0) (void)tc::mbar_wait(&full[st], (unsigned)(last_issued[st] / stages) & 1u);
+    }
+    __syncwarp();
+    __syncthreads();
+    return;
+  }
+
+  // ---------------- consumer warps: pairs of tasks, pair index % 8 == warp
+  int u = 0, pair0 = 0;
+  for (int c = c_lo; c < c_hi; ++c) {
+    const int n = hist[c];
+    if (n == 0) continue;
+    const int st = u % stages;
+    if (!tc::mbar_wait(&full[st], (unsigned)(u / stages) & 1u)) {
+      misc[2] = 1;
+      break;
+    }
+    if (u == 0) RDL_TRACE_POINT(3, 3);
+    const uint32_t kst = smem_u32(ring + st * AT_STAGE_BYTES), vst = kst + 16384;
+    const int tbeg = pre[c] - n - lbase, npair = (n + 1) / 2;
+    int pfirst = (warp - pair0 % AT_CONS + AT_CONS) % AT_CONS;
+    for (int pp = pfirst; pp < npair; pp += AT_CONS) {
+      const int tA = list[tbeg + 2 * pp];
+      const bool hasB = 2 * pp + 1 < n;
+      const int tB = hasB ? list[tbeg + 2 * pp + 1] : tA;
+      const int iA = tA >> 8, iB = tB >> 8;
+      // ---- S = Q K^T for rows (iA heads 0-7, iB heads 0-7) x 64 keys
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      {
+        const int mi = lane >> 3;
+        const uint32_t qrow = smem_u32(qs + ((mi & 1) ? iB : iA) * 2048) + (lane & 7) * 256;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t a[4];
+          const int uq = 2 * ks + (mi >> 1);
+          ldsm_x4(qrow + ((uq ^ (lane & 7)) << 4), a[0], a[1], a[2], a[3]);
+#pragma unroll
+          for (int np = 0; np < 4; ++np) {
+            uint32_t b0, b1, b2, b3;
+            const int key = 16 * np + 8 * (mi >> 1) + (lane & 7), col = 16 * ks + 8 * (mi & 1);
+            ldsm_x4(kst + kv_off(key, col), b0, b1, b2, b3);
+            mma_bf16(sc[2 * np], a, b0, b1);
+            mma_bf16(sc[2 * np + 1], a, b2, b3);
+          }
+        }
+      }
+      // ---- per-row mask and softmax (row gq: task A, row gq + 8: task B)
+      const bool winA = (tA & TASK_WIN) != 0, winB = (tB & TASK_WIN) != 0;
+      const int pA = pos_s[iA], pB = pos_s[iB];
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = 8 * nt + 2 * tq + (e & 1);
+          const bool hb = e >= 2;
+          const bool win = hb ? winB : winA;
+          const int p = hb ? pB : pA;
+          const int j2 = S * c + key;
+          const bool in = win ? (j2 >= p - w && j2 <= p + w) : key < CONTENT;
+          const float v = in ? sc[nt][e] * sl2 : -INFINITY;
+          sc[nt][e] = v;
+          mx[hb] = fmaxf(mx[hb], v);
+        }
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        mx[hb] = fmaxf(mx[hb], __shfl_xor_sync(0xffffffffu, mx[hb], 1));
+        mx[hb] = fmaxf(mx[hb], __shfl_xor_sync(0xffffffffu, mx[hb], 2));
+      }
+      float sm[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int hb = e >> 1;
+          const float pv = fast_exp2(sc[nt][e] - mx[hb]);   // masked: exp2(-inf) = 0
+          sc[nt][e] = pv;
+          sm[hb] += pv;
+        }
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 1);
+        sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 2);
+      }
+      // chunk tasks are normalised here; window tasks keep (max, sum) for the merge
+      const float fA = winA ? 1.f : 1.f / sm[0], fB = winB ? 1.f : 1.f / sm[1];
+      // P as bf16 A fragments (FA2 layout: the S accumulators of n-tiles 2kk, 2kk+1)
+      uint32_t pa[4][4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        pa[kk][0] = pack_bf16(sc[2 * kk][0] * fA, sc[2 * kk][1] * fA);
+        pa[kk][1] = pack_bf16(sc[2 * kk][2] * fB, sc[2 * kk][3] * fB);
+        pa[kk][2] = pack_bf16(sc[2 * kk + 1][0] * fA, sc[2 * kk + 1][1] * fA);
+        pa[kk][3] = pack_bf16(sc[2 * kk + 1][2] * fB, sc[2 * kk + 1][3] * fB);
+      }
+      float* dstA = nullptr;
+      float* dstB = nullptr;
+      {
+        const int slotA = tA & 127, slotB = tB & 127;
+        const size_t rgA = (size_t)(b * Lq + iA) * Hkv + g, rgB = (size_t)(b * Lq + iB) * Hkv + g;
+        if (gq < G) {
+          dstA = (tA & TASK_WIN) ? ow_part + ((rgA * nwt + slotA) * G + gq) * D : o_part + ((rgA * K + slotA) * G + gq) * D;
+          if (hasB)
+            dstB = (tB & TASK_WIN) ? ow_part + ((rgB * nwt + slotB) * G + gq) * D : o_part + ((rgB * K + slotB) * G + gq) * D;
+          if (tq == 0 && (tA & TASK_WIN)) ml_part[(rgA * nwt + slotA) * G + gq] = make_float2(mx[0] * LN2, sm[0]);
+          if (tq == 0 && hasB && (tB & TASK_WIN)) ml_part[(rgB * nwt + slotB) * G + gq] = make_float2(mx[1] * LN2, sm[1]);
+        }
+      }
+      // ---- O = P V, 64 dims at a time
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float oc[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) oc[nt][0] = oc[nt][1] = oc[nt][2] = oc[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int mi = lane >> 3;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            uint32_t b0, b1, b2, b3;
+            const int key = 16 * kk + 8 * (mi & 1) + (lane & 7), col = 64 * half + 16 * m + 8 * (mi >> 1);
+            ldsm_x4_t(vst + kv_off(key, col), b0, b1, b2, b3);
+            mma_bf16(oc[2 * m], pa[kk], b0, b1);
+            mma_bf16(oc[2 * m + 1], pa[kk], b2, b3);
+          }
+        }
+        if (dstA) {
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+            *reinterpret_cast<float2*>(dstA + 64 * half + 8 * nt + 2 * tq) = make_float2(oc[nt][0], oc[nt][1]);
+        }
+        if (dstB) {
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+            *reinterpret_cast<float2*>(dstB + 64 * half + 8 * nt + 2 * tq) = make_float2(oc[nt][2], oc[nt][3]);
+        }
+      }
+    }
+    if (u == 0) RDL_TRACE_POINT(3, 7);
+    pair0 += npair;
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&empty[st]);
+    ++u;
+  }
+  __syncthreads();   // pairs with the producer's final barrier
+  RDL_TRACE_POINT(3, 5);
+}
+
+// =====================================================================================
+// dec_comb_kernel: one warp per (b, i, h); lane l owns dims 4l .. 4l+3.  Merges the
+// window slab partials (max, sum, unnormalised vector) and, on route layers, the chunk
+// outputs with weights e^{z_c}: one partition, o = sum(weight * vector) / sum(weight).
+// Parts are loaded in batches before their weights are known (unused loads are harmless).
+// =====================================================================================
+template <bool ROUTE>
+__global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict__ q_pos,
+                                                       const int32_t* __restrict__ idx,
+                                                       const float* __restrict__ z_sel,
+                                                       const float* __restrict__ o_part,
+                                                       const float* __restrict__ ow_part,
+                                                       const float2* __restrict__ ml_part, int B, int L, int Lq,
+                                                       int Hq, int Hkv, int K, int w, int flags,
+                                                       __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  constexpr int D = 128;
+  grid_dep_wait();
+  grid_dep_launch();
+  RDL_TRACE_POINT(4, 1);
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (item >= (long long)B * Lq * Hq) return;
+  const int h = (int)(item % Hq);
+  const int i = (int)((item / Hq) % Lq);
+  const int b = (int)(item / ((long long)Hq * Lq));
+  const int C = L / S, G = Hq / Hkv, g = h / G, hl = h % G;
+  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+  if (ROUTE && is_mask_slot(p)) return;
+  const int nwt = max_win_slabs(w);
+  const int nw = w >= 0 ? win_hi(p, w, L) - win_lo(p, w) + 1 : 0;
+  const size_t rg = (size_t)(b * Lq + i) * Hkv + g;
+  // window slabs: lanes s, s + 32 hold slab s's (max, sum)
+  float wm[2] = {-INFINITY, -INFINITY}, wl[2] = {0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int s2 = lane + 32 * u;
+    if (s2 < nw) {
+      const float2 ml = ml_part[(rg * nwt + s2) * G + hl];
+      wm[u] = ml.x;
+      wl[u] = ml.y;
+    }
+  }
+  float4 vw[12];
+#pragma unroll
+  for (int s2 = 0; s2 < 12; ++s2)
+    vw[s2] = s2 < nw ? *reinterpret_cast<const float4*>(ow_part + ((rg * nwt + s2) * G + hl) * D + 4 * lane)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+  // chunk slots: lanes k, k+32 hold slot k's logit (-inf when empty or skipped)
+  float zk[2] = {-INFINITY, -INFINITY};
+  if (ROUTE) {
+    const int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
+    const float* zrow = z_sel + ((size_t)(b * Hq + h) * Lq + i) * K;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      if (k < K) {
+        const int c = irow[k];
+        bool ok = c >= 0 && c < C;
+        if (ok && (flags & RDL_FLAG_CHECKS) && !chunk_eligible(c, p, w)) ok = false;
+        if (ok) zk[u] = zrow[k];
+      }
+    }
+  }
+  float M = fmaxf(fmaxf(wl[0] > 0.f ? wm[0] : -INFINITY, wl[1] > 0.f ? wm[1] : -INFINITY), fmaxf(zk[0], zk[1]));
+  M = warp_max(M);
+  if (M == -INFINITY) M = 0.f;
+  const float ew0 = wl[0] > 0.f ? expf(wm[0] - M) : 0.f;     // slab weights e^{m - M}
+  const float ew1 = wl[1] > 0.f ? expf(wm[1] - M) : 0.f;
+  const float ek0 = zk[0] == -INFINITY ? 0.f : expf(zk[0] - M);
+  const float ek1 = zk[1] == -INFINITY ? 0.f : expf(zk[1] - M);
+  const float Zs = warp_sum(ew0 * wl[0] + ew1 * wl[1] + ek0 + ek1);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s2 = 0; s2 < 12; ++s2) {
+    const float f = __shfl_sync(0xffffffffu, ew0, s2);
+    if (s2 < nw && f != 0.f) {
+      acc.x += f * vw[s2].x; acc.y += f * vw[s2].y; acc.z += f * vw[s2].z; acc.w += f * vw[s2].w;
+    }
+  }
+  for (int s2 = 12; s2 < nw; ++s2) {
+    const float f = __shfl_sync(0xffffffffu, s2 < 32 ? ew0 : ew1, s2 & 31);
+    const float4 v = *reinterpret_cast<const float4*>(ow_part + ((rg * nwt + s2) * G + hl) * D + 4 * lane);
+    if (f != 0.f) {
+      acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
+    }
+  }
+  if (ROUTE) {
+    const float* pbase = o_part + (rg * K * G + hl) * D + 4 * lane;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = k0 + u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)(k0 + u) * G * D)
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int k = k0 + u;
+        const float f = __shfl_sync(0xffffffffu, (k < 32) ? ek0 : ek1, k & 31);
+        if (k < K && f != 0.f) {
+          acc.x += f * v[u].x; acc.y += f * v[u].y; acc.z += f * v[u].z; acc.w += f * v[u].w;
+        }
+      }
+    }
+  }
+  const float inv = Zs > 0.f ? 1.f / Zs : 0.f;
+  __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + h) * D + 4 * lane;
+  const __nv_bfloat162 o01 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 o23 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&o01);
+  pk.y = *reinterpret_cast<const uint32_t*>(&o23);
+  *reinterpret_cast<uint2*>(orow) = pk;
+  if (lse && lane == 0) lse[(size_t)(b * Hq + h) * Lq + i] = Zs > 0.f ? M + logf(Zs) : -INFINITY;
+}
+
+}  // namespace dec
+}  // namespace rdl

@@ -443,41 +443,16 @@ __device__ __forceinline__ int block_excl_scan256(int v, int* warp_sums, int& to
   return base + x - v;
 }
 
-// One CTA (256 threads) per (b, g, i): the same exact top-K as topk_radix_kernel, for few
-// rows over many chunks (decode blocks).  Keys are split across the CTA; the selection is
-// compacted in chunk order with block scans.
-__global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ zeta,
-                                                       const float* __restrict__ z_all,
-                                                       const int32_t* __restrict__ q_pos, int Lq, int L,
-                                                       int Hq, int Hkv, int K, int32_t* __restrict__ idx,
-                                                       float* __restrict__ z_sel) {
-  extern __shared__ uint32_t tc_keys[];
-  __shared__ unsigned hist[256];
-  __shared__ int warp_sums[8];
-  __shared__ int sel_s[64];
-  __shared__ int bc[3];
-  const int C = L / S, G = Hq / Hkv;
+// Exact top-K of the order keys keys[0..C) by one CTA of 256 threads: a 4-pass 8-bit radix
+// select for the K-th largest key, then an in-order compaction that takes every key above it
+// and the first (by chunk index) of the keys equal to it.  sel_s receives the selected
+// chunk indices in ascending order; returns how many there are (min(#valid, K)).
+__device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int K, unsigned* hist,
+                                               unsigned (*whist)[256], int* warp_sums, int* bc, int* sel_s) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int item = blockIdx.x, b = blockIdx.y;
-  const int g = item / Lq, i = item % Lq;
-  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
-  int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
-  if (is_mask_slot(p)) {
-    for (int e = tid; e < K * G; e += 256) {
-      const int k = e % K, hl = e / K;
-      if (hl == 0) irow[k] = -1;
-      z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
-    }
-    return;
-  }
-  const float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
   const uint32_t kneg = order_key(-INFINITY);
   int nv = 0;
-  for (int c = tid; c < C; c += 256) {
-    const uint32_t k = order_key(zr[c]);
-    tc_keys[c] = k;
-    nv += k > kneg;
-  }
+  for (int c = tid; c < C; c += 256) nv += keys[c] > kneg;
   int nvalid;
   (void)block_excl_scan256(nv, warp_sums, nvalid);
   uint32_t thr = kneg;
@@ -486,33 +461,47 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
     uint32_t prefix = 0, pmask = 0;
     need = K;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      hist[tid] = 0;
-      __syncthreads();
+      // per-warp histograms: no two warps contend for one bin (the keys cluster in a few
+      // digits, so a shared histogram would serialise the whole CTA on those bins)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) whist[warp][lane * 8 + u] = 0;
+      __syncwarp();
       for (int base = 0; base < C; base += 256) {
         const int c = base + tid;
-        const uint32_t k = c < C ? tc_keys[c] : 0u;
-        const bool in = c < C && (k & pmask) == prefix;
-        const unsigned dig = in ? ((k >> shift) & 255u) : 256u;
-        const unsigned peers = __match_any_sync(0xffffffffu, dig);
-        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+        const uint32_t k = c < C ? keys[c] : 0u;
+        if (c < C && (k & pmask) == prefix) atomicAdd(&whist[warp][(k >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      __syncthreads();
+      {
+        unsigned sum = 0;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) sum += whist[w8][tid];
+        hist[tid] = sum;
       }
       __syncthreads();
       if (warp == 0) {
-        int local = 0;
+        // lane l owns bins 255-8l .. 248-8l (largest digits first); an inclusive warp scan
+        // of the lane counts finds the lane holding the need-th largest key
+        int cnt[8], local = 0;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) local += (int)hist[lane * 8 + u];
-        int incl = 0, tl = -1, excl = 0;
-        for (int l2 = 31; l2 >= 0; --l2) {
-          const int v = __shfl_sync(0xffffffffu, local, l2);
-          if (tl < 0 && incl + v >= need) { tl = l2; excl = incl; }
-          incl += v;
+        for (int u = 0; u < 8; ++u) {
+          cnt[u] = (int)hist[255 - 8 * lane - u];
+          local += cnt[u];
         }
-        if (lane == tl) {
-          int run = excl, dg = 0, ca = excl;
-          for (int u = 7; u >= 0; --u) {
-            const int v = (int)hist[lane * 8 + u];
-            if (run + v >= need) { dg = lane * 8 + u; ca = run; break; }
-            run += v;
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+        if (lane == __ffs(hit) - 1) {
+          int run = incl - local, dg = 0, ca = run;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (run + cnt[u] >= need) { dg = 255 - 8 * lane - u; ca = run; break; }
+            run += cnt[u];
           }
           bc[0] = dg;
           bc[1] = ca;
@@ -530,7 +519,7 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
   const int seg = (C + 255) / 256, c0 = tid * seg, c1 = min(C, c0 + seg);
   int ngt = 0, nties = 0;
   for (int c = c0; c < c1; ++c) {
-    const uint32_t k = tc_keys[c];
+    const uint32_t k = keys[c];
     ngt += k > thr;
     nties += (need > 0 && k == thr);
   }
@@ -540,14 +529,48 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
   const int pos0 = block_excl_scan256(ngt + take_ties, warp_sums, tot);
   int pos = pos0, tk = 0;
   for (int c = c0; c < c1; ++c) {
-    const uint32_t k = tc_keys[c];
+    const uint32_t k = keys[c];
     bool take = k > thr;
     if (!take && need > 0 && k == thr && tk < take_ties) { take = true; ++tk; }
     if (take && pos < K) sel_s[pos] = c;
     pos += take;
   }
   __syncthreads();
-  const int nsel = min(tot, K);
+  return min(tot, K);
+}
+
+// One CTA (256 threads) per (b, g, i): the same exact top-K as topk_radix_kernel, for few
+// rows over many chunks (decode blocks).  Keys are split across the CTA; the selection is
+// compacted in chunk order with block scans.
+__global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ zeta,
+                                                       const float* __restrict__ z_all,
+                                                       const int32_t* __restrict__ q_pos, int Lq, int L,
+                                                       int Hq, int Hkv, int K, int32_t* __restrict__ idx,
+                                                       float* __restrict__ z_sel) {
+  extern __shared__ uint32_t tc_keys[];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned whist[8][256];
+  __shared__ int warp_sums[8];
+  __shared__ int sel_s[64];
+  __shared__ int bc[3];
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x;
+  const int item = blockIdx.x, b = blockIdx.y;
+  const int g = item / Lq, i = item % Lq;
+  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
+  int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
+  if (is_mask_slot(p)) {
+    for (int e = tid; e < K * G; e += 256) {
+      const int k = e % K, hl = e / K;
+      if (hl == 0) irow[k] = -1;
+      z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
+    }
+    return;
+  }
+  const float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
+  for (int c = tid; c < C; c += 256) tc_keys[c] = order_key(zr[c]);
+  __syncthreads();
+  const int nsel = cta_select_topk(tc_keys, C, K, hist, whist, warp_sums, bc, sel_s);
   for (int e = tid; e < K * G; e += 256) {
     const int k = e % K, hl = e / K, h = g * G + hl;
     const int c = k < nsel ? sel_s[k] : -1;

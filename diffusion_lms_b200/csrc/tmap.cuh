@@ -70,3 +70,22 @@ inline bool make_tmap_q_run(CUtensorMap* map, const void* base, unsigned long lo
 }
 
 }  // namespace rdl
+
+namespace rdl {
+
+// Summaries s [rows, 128] fp32 (row stride 512 B) viewed as (32 columns, rows, 4 slices):
+// one box of box_rows rows lands as 4 slices [box_rows][128 B] (columns 0-31, 32-63, ...),
+// each with the 128-byte swizzle.  Rows past the end read as zeros.
+inline bool make_tmap_f32_rows(CUtensorMap* map, const void* base, unsigned long long rows, unsigned box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {32, rows, 4};
+  cuuint64_t strides[2] = {512, 128};
+  cuuint32_t box[3] = {32, box_rows, 4};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace rdl

@@ -24,7 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_DEVICE_CHECK = \
     0, -1, -2, -3, -4, -5, -6
 ERR_SCRATCH_LIMIT = -7
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 BF16, F32 = 0, 1
 FLAG_MEAN_SUMMARY, FLAG_CHECKS = 0x1, 0x2
 WS_SCORE, WS_ATTN, WS_SWA = 0, 1, 2

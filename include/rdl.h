@@ -164,10 +164,11 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * entry point takes the same arguments as rdl_route_attn minus the workspace and uses a
  * static scratch array that librdl.so itself holds in device memory instead.
  *
- * Scratch limit: RDL_NOALLOC_SCRATCH_BYTES (16 MiB) per device, reserved on every GPU
+ * Scratch limit: RDL_NOALLOC_SCRATCH_BYTES (32 MiB) per device, reserved on every GPU
  * that loads the library, until the process exits.  A call whose
  * rdl_workspace_bytes(RDL_WS_ATTN, dims, dtype) exceeds it returns RDL_ERR_SCRATCH_LIMIT
- * and launches nothing (a 32-query decode block over 28 heads needs about 11.5 MiB).
+ * and launches nothing (a 32-query decode block over 28 heads with K = 32 and a +-256 window
+ * needs about 18.5 MiB).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture begins.
  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
@@ -175,7 +176,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * it needs to start at zero.  Calls that overlap on the GPU (concurrent streams, or
  * several host threads) race on the array: serialise them.
  */
-#define RDL_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define RDL_NOALLOC_SCRATCH_BYTES (32u << 20)
 rdl_status rdl_route_attn_noalloc(const void* q, const int32_t* q_pos, const void* k,
                                   const void* v, const int32_t* idx, const float* z_sel,
                                   const rdl_dims* dims, rdl_dtype dtype, void* o, float* lse,

@@ -125,6 +125,27 @@ def test_device_checks_record_without_fault():
     assert rdl.rdl_last_device_status() == rdl.OK          # cleared on read
 
 
+def test_decode_device_checks_record_without_fault():
+    """Decode-block kernels: a chunk id beyond C and one inside the row's window are recorded
+    in the status word and skipped; every output stays finite."""
+    wl = W.make_inputs(small(L=8192, Lq=32, K=32, w=256), seed=17, n_needles=4, decode_block=32)
+    inp = api.to_device(wl)
+    inp.dims.flags = rdl.FLAG_CHECKS
+    out = api.alloc_outputs(inp.dims, inp.dtype)
+    api.summary_pool(inp, out)
+    api.score_topk(inp, out)
+    api.route_attn(inp, out)
+    torch.cuda.synchronize()
+    assert rdl.rdl_last_device_status() == rdl.OK
+    own = int(inp.q_pos[0, 6].item()) // 64
+    out.idx[0, 0, 5, 0] = 10_000
+    out.idx[0, 1, 6, 1] = own
+    api.route_attn(inp, out)
+    assert rdl.rdl_last_device_status() == rdl.ERR_DEVICE_CHECK
+    assert rdl.rdl_last_device_status() == rdl.OK
+    assert torch.isfinite(out.o.float()).all()
+
+
 def test_bitwise_repeatable():
     for dm, dec in ((small(), 0), (small(L=8192, Lq=32, K=32, w=256), 32)):
         wl = W.make_inputs(dm, seed=18, n_needles=4, decode_block=dec)
