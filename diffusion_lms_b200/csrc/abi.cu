@@ -322,7 +322,7 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
     return RDL_ERR_CUDA;
   const float tau = (float)(1.0 / sqrt((double)dm->d));
   // launched early only behind dec_t_kernel: its prologue loads inputs before the wait
-  if (launch_ex(res, kern, dim3(gr.ranges, dm->Hq, dm->B), dim3(256), gr.smem, st, smap, summary,
+  if (launch_ex(res, kern, dim3(gr.ranges, dm->Hq, dm->B), dim3(dec::SC_WARPS * 32), gr.smem, st, smap, summary,
                  static_cast<const __nv_bfloat16*>(q), q_pos, (const float*)(res ? t : nullptr),
                  static_cast<const __nv_bfloat16*>(w_up), entropy, dm->Lq, dm->L, dm->Hq, res ? dm->r : 0, dm->w, tau,
                  dm->lambda, gr.ncr, gr.boxr, gr.nbox, gr.nstg, z_all) != cudaSuccess)
@@ -330,12 +330,12 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
   const int G = dm->Hq / dm->Hkv;
   const bool zs = C % 4 == 0 && G * C <= dec::DK_MAXZ;
   const size_t ksm = (size_t)(((C + 3) & ~3) + (zs ? G * C : 0)) * sizeof(uint32_t);
-  auto tk = C <= 1024 ? (zs ? dec::dec_topk_kernel<true, 4> : dec::dec_topk_kernel<false, 4>)
-            : C <= 2048 ? (zs ? dec::dec_topk_kernel<true, 8> : dec::dec_topk_kernel<false, 8>)
-                        : (zs ? dec::dec_topk_kernel<true, 32> : dec::dec_topk_kernel<false, 32>);
+  auto tk = C <= 1024 ? (zs ? dec::dec_topk_kernel<true, 2> : dec::dec_topk_kernel<false, 2>)
+            : C <= 2048 ? (zs ? dec::dec_topk_kernel<true, 4> : dec::dec_topk_kernel<false, 4>)
+                        : (zs ? dec::dec_topk_kernel<true, 16> : dec::dec_topk_kernel<false, 16>);
   if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksm) != cudaSuccess)
     return RDL_ERR_CUDA;
-  if (launch_pdl(tk, dim3(dm->Lq, dm->Hkv, dm->B), dim3(256), ksm, st, (const float*)z_all, q_pos, dm->Lq, dm->L,
+  if (launch_pdl(tk, dim3(dm->Lq, dm->Hkv, dm->B), dim3(dec::DK_THREADS), ksm, st, (const float*)z_all, q_pos, dm->Lq, dm->L,
                  dm->Hq, dm->Hkv, dm->K, idx, z_sel) != cudaSuccess)
     return RDL_ERR_CUDA;
   return RDL_OK;

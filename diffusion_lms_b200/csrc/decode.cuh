@@ -178,17 +178,20 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
 }
 
 // =====================================================================================
-// dec_score_kernel: CTA = (chunk range, query head h, batch b); 8 warps.
+// dec_score_kernel: CTA = (chunk range, query head h, batch b); 16 warps.
 // MT = m-tiles of 16 query rows (rows = Lq <= 16*MT).
 // Shared memory:
 //   ring   nstg stages of boxr summary rows, each [4 slices][boxr][32 fp32] with the
-//          128-byte swizzle of the TMA box (16-byte unit ^ row % 8)
+//          128-byte swizzle of the TMA box (16-byte unit ^ row % 8); rewritten in place to
+//          bf16 hi/lo terms once landed
 //   wup    W_up columns of head h: [r][128] bf16, unit-swizzled (ldmatrix.trans)
 //   qh     q rows of head h: [16*MT][136] bf16 (padded rows)
-//   qt     q_res rows: [16*MT][132] fp32 (padded rows)
+//   qsp    q_res rows split into bf16 hi/lo: [16*MT][hi 128 | lo 128], unit-swizzled
+//   ts     t rows: [16*MT][r + 8] fp32
 // =====================================================================================
+constexpr int SC_WARPS = 16;
 struct ScoreSmem {
-  int ring, wup, qh, qt, ts, hs, ps, bar, total;
+  int ring, wup, qh, qsp, ts, hs, ps, bar, total;
 };
 __host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nstg, int ncr) {
   ScoreSmem s{};
@@ -196,7 +199,7 @@ __host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nst
   s.ring = off; off += nstg * boxr * 512;
   s.wup = off;  off += (r > 0 ? r : 1) * 256;
   s.qh = off;   off += MT * 16 * 272;
-  s.qt = off;   off += MT * 16 * 528;
+  s.qsp = off;  off += MT * 16 * 512;
   s.ts = off;   off += MT * 16 * (r + 8) * 4;
   s.hs = off;   off += ((ncr + 3) / 4) * 16;
   s.ps = off;   off += 64 * 4;
@@ -205,31 +208,34 @@ __host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nst
   return s;
 }
 
+// byte offset of 16-byte unit u (0..31: hi 0-15, lo 16-31) of row `row` in a qsp tile
+__device__ __forceinline__ uint32_t qsp_off(int row, int u) { return (uint32_t)(row * 512 + ((u ^ (row & 7)) << 4)); }
+
 template <int MT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(SC_WARPS * 32, 1)
     dec_score_kernel(const __grid_constant__ CUtensorMap smap, const float* __restrict__ smap_base,
-                     const __nv_bfloat16* __restrict__ q,
-                     const int32_t* __restrict__ q_pos, const float* __restrict__ t,
-                     const __nv_bfloat16* __restrict__ w_up, const float* __restrict__ entropy, int Lq, int L,
-                     int Hq, int r, int w, float tau, float lambda, int ncr, int boxr, int nbox, int nstg,
-                     float* __restrict__ z_all) {
+                     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
+                     const float* __restrict__ t, const __nv_bfloat16* __restrict__ w_up,
+                     const float* __restrict__ entropy, int Lq, int L, int Hq, int r, int w, float tau,
+                     float lambda, int ncr, int boxr, int nbox, int nstg, float* __restrict__ z_all) {
   constexpr int D = 128;
-  constexpr int NG = 8 / MT;                  // warps per m-tile (n-groups)
+  constexpr int NT = SC_WARPS * 32;
+  constexpr int NG = SC_WARPS / MT;           // warps per m-tile (n-groups)
   extern __shared__ unsigned char sc_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sc_raw) + 1023) & ~uintptr_t(1023));
   const ScoreSmem L_ = score_smem(MT, r, boxr, nstg, ncr);
   unsigned char* ring = base + L_.ring;
   unsigned char* wup = base + L_.wup;
   unsigned char* qh = base + L_.qh;
-  float* qt = reinterpret_cast<float*>(base + L_.qt);
+  unsigned char* qsp = base + L_.qsp;
   float* ts = reinterpret_cast<float*>(base + L_.ts);
   float* hs = reinterpret_cast<float*>(base + L_.hs);
   int* ps = reinterpret_cast<int*>(base + L_.ps);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + L_.bar);
+  RDL_TRACE_POINT(1, 0);
 
   const int C = L / S;
   const int b = blockIdx.z, h = blockIdx.y;
-  RDL_TRACE_POINT(1, 0);
   const int c0 = blockIdx.x * ncr, c1 = min(C, c0 + ncr);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
@@ -243,7 +249,7 @@ __global__ void __launch_bounds__(256, 1)
   // ---- prologue: only TMA and cp.async.cg loads of inputs (no kernel of this call writes
   // them, and this kernel is launched early only behind dec_t_kernel, which has waited)
   if (tid == 0) {
-    for (int s = 0; s < nstg; ++s) tc::mbar_init(&full[s], 1);
+    for (int st = 0; st < nstg; ++st) tc::mbar_init(&full[st], 1);
     tc::mbar_fence_init();
   }
   __syncthreads();
@@ -253,22 +259,22 @@ __global__ void __launch_bounds__(256, 1)
       tc::tma_load_3d(ring + bx * boxr * 512, &smap, 0, (int)(srow0 + (size_t)bx * boxr), 0, &full[bx]);
     }
   }
-  for (int e = tid; e < r * 16; e += 256) {
+  for (int e = tid; e < r * 16; e += NT) {
     const int kk = e >> 4, u = e & 15;
     cp_async16(smem_u32(wup + kk * 256 + ((u ^ (kk & 7)) << 4)), w_up + (size_t)kk * Hq * D + h * D + u * 8);
   }
-  for (int e = tid; e < Lq * 16; e += 256) {
+  for (int e = tid; e < Lq * 16; e += NT) {
     const int i = e >> 4, u = e & 15;
     cp_async16(smem_u32(qh + i * 272 + u * 16), q + ((size_t)(b * Lq + i) * Hq + h) * D + u * 8);
   }
   cp_async_commit();
-  for (int j = tid; j < c1 - c0; j += 256) hs[j] = __ldcg(entropy + (size_t)(b * Hq + h) * C + c0 + j);
+  for (int j = tid; j < c1 - c0; j += NT) hs[j] = __ldcg(entropy + (size_t)(b * Hq + h) * C + c0 + j);
   if (tid < MT * 16) ps[tid] = tid < Lq ? (q_pos ? __ldcg(q_pos + (size_t)b * Lq + tid) : tid) : INT_MIN;
   // rows beyond the ring: pulled into L2 now, loaded into the ring when a stage frees
-  for (int bx = nstg + (tid >> 5); bx < nb; bx += 8) {
+  for (int bx = nstg + warp; bx < nb; bx += SC_WARPS) {
     const char* src = reinterpret_cast<const char*>(smap_base) + (srow0 + (size_t)bx * boxr) * 512;
     const int bytes = min(boxr, (c1 - c0) - bx * boxr) * 512;
-    for (int off = (tid & 31) * 4096; off < bytes; off += 32 * 4096)
+    for (int off = lane * 4096; off < bytes; off += 32 * 4096)
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src + off), "r"(min(4096, bytes - off))
                    : "memory");
   }
@@ -278,14 +284,15 @@ __global__ void __launch_bounds__(256, 1)
   RDL_TRACE_POINT(1, 1);
   if (r > 0) {
     const int nu = r / 4;                       // 16-byte units per t row
-    for (int e = tid; e < Lq * nu; e += 256) {
+    for (int e = tid; e < Lq * nu; e += NT) {
       const int i = e / nu, u = e % nu;
       cp_async16(smem_u32(ts + i * (r + 8) + u * 4), t + (size_t)(b * Lq + i) * r + u * 4);
     }
   }
   cp_async_commit();
 
-  // ---- q_res = q + t W_up for this warp's m-tile and n-group (tensor cores, t split)
+  // ---- q_res = q + t W_up for this warp's m-tile and n-group (tensor cores, t split),
+  // written straight into the split hi/lo tile
   {
     constexpr int NPW = 16 / NG;              // n-tiles (of 8 columns) per warp
     float ua[NPW][4];
@@ -327,45 +334,43 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int row = mw * 16 + gq + 8 * hr;
-        const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162*>(qh + row * 272 + col * 2);
-        const float2 qf = __bfloat1622float2(qv);
-        qt[row * 132 + col] = qf.x + ua[n][2 * hr];
-        qt[row * 132 + col + 1] = qf.y + ua[n][2 * hr + 1];
+        const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qh + row * 272 + col * 2));
+        uint32_t hi, lo;
+        split2(qf.x + ua[n][2 * hr], qf.y + ua[n][2 * hr + 1], hi, lo);
+        // unit col/8 holds columns col/8*8 .. +7; this pair is word (col % 8) / 2 of it
+        *reinterpret_cast<uint32_t*>(qsp + qsp_off(row, col >> 3) + (col & 7) * 2) = hi;
+        *reinterpret_cast<uint32_t*>(qsp + qsp_off(row, 16 + (col >> 3)) + (col & 7) * 2) = lo;
       }
     }
   }
   __syncthreads();
-  // ---- A fragments of q_res (hi/lo) for this warp's m-tile, all 8 k-steps
-  uint32_t ahi[8][4], alo[8][4];
-  {
-    const int row0 = mw * 16 + gq, row1 = row0 + 8;
+  RDL_TRACE_POINT(1, 3);
+  int wlo[2], whi[2];   // window chunk range of the warp's two rows: chunks wlo..whi are not eligible
+  const int irow[2] = {mw * 16 + gq, mw * 16 + gq + 8};
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int ca = 16 * ks + 2 * tq;
-      const float2 v0 = *reinterpret_cast<const float2*>(qt + row0 * 132 + ca);
-      const float2 v1 = *reinterpret_cast<const float2*>(qt + row1 * 132 + ca);
-      const float2 v2 = *reinterpret_cast<const float2*>(qt + row0 * 132 + ca + 8);
-      const float2 v3 = *reinterpret_cast<const float2*>(qt + row1 * 132 + ca + 8);
-      split2(v0.x, v0.y, ahi[ks][0], alo[ks][0]);
-      split2(v1.x, v1.y, ahi[ks][1], alo[ks][1]);
-      split2(v2.x, v2.y, ahi[ks][2], alo[ks][2]);
-      split2(v3.x, v3.y, ahi[ks][3], alo[ks][3]);
+  for (int hr = 0; hr < 2; ++hr) {
+    const int p = ps[irow[hr]];
+    if (w < 0 || p == INT_MIN) {
+      wlo[hr] = 1;
+      whi[hr] = 0;
+    } else {
+      wlo[hr] = p - w <= 0 ? INT_MIN : (p - w) / S;     // chunk containing p - w (or none below 0)
+      whi[hr] = (p + w) / S;
     }
   }
-  const int prow[2] = {ps[mw * 16 + gq], ps[mw * 16 + gq + 8]};
-  RDL_TRACE_POINT(1, 3);
-  const int irow[2] = {mw * 16 + gq, mw * 16 + gq + 8};
   // ---- scores over the range, box by box as the TMA loads land.  Each landed box is first
   // rewritten in place: every 128-byte segment (32 fp32 of one summary row) becomes 32 bf16
   // hi terms (logical 16-byte units 0-3) and 32 bf16 lo terms (units 4-7), x = hi + lo to
   // ~2^-17, keeping the unit ^ (row % 8) swizzle so the fragment loads stay conflict-free.
   const int ntb = boxr / 8;
   for (int bx = 0; bx < nb; ++bx) {
-    const int s = bx % nstg;
-    if (!tc::mbar_wait(&full[s], (unsigned)(bx / nstg) & 1u)) break;
+    const int st = bx % nstg;
+    if (!tc::mbar_wait(&full[st], (unsigned)(bx / nstg) & 1u)) break;
     if (bx == 0) RDL_TRACE_POINT(1, 4);
-    unsigned char* stg = ring + s * boxr * 512;
-    for (int seg = tid; seg < 4 * boxr; seg += 256) {
+    if (bx == 1) RDL_TRACE_POINT(1, 6);
+    if (bx == nb - 1) RDL_TRACE_POINT(1, 7);
+    unsigned char* stg = ring + st * boxr * 512;
+    for (int seg = tid; seg < 4 * boxr; seg += NT) {
       const int rr = seg % boxr;
       unsigned char* sp = stg + (seg / boxr) * boxr * 128 + rr * 128;
       const int sw = rr & 7;
@@ -386,47 +391,67 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     __syncthreads();
-    const uint32_t st = smem_u32(stg);
+    const uint32_t stu = smem_u32(stg);
     const int cb = c0 + bx * boxr;
-    for (int nt = ng; nt < ntb; nt += NG) {
-      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
-      const int rl = nt * 8 + (lane & 7), mj = lane >> 3;
+    // this warp's n-tiles of the box: ng, ng + NG, ... (at most 2 for NG >= ntb / 2)
+    for (int nt0 = ng; nt0 < ntb; nt0 += 2 * NG) {
+      const int nt1 = nt0 + NG;
+      const bool two = nt1 < ntb;
+      float a0[2][4], a1[2][4], a2[2][4];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a0[x][e] = a1[x][e] = a2[x][e] = 0.f;
+      const int mj = lane >> 3;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        // matrices: hi dims d0..+7, hi d0+8..+15, lo d0..+7, lo d0+8..+15 of chunk rows nt*8..+7
+        uint32_t ahi[4], alo[4];
+        const int ra = mw * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), ua = 2 * ks + (lane >> 4);
+        ldsm_x4(smem_u32(qsp + qsp_off(ra, ua)), ahi[0], ahi[1], ahi[2], ahi[3]);
+        ldsm_x4(smem_u32(qsp + qsp_off(ra, 16 + ua)), alo[0], alo[1], alo[2], alo[3]);
         const int un = (mj >= 2 ? 4 : 0) + ((16 * ks) & 31) / 8 + (mj & 1);
-        uint32_t bh0, bh1, bl0, bl1;
-        ldsm_x4(st + (ks >> 1) * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
-        mma_bf16(a0, ahi[ks], bh0, bh1);
-        mma_bf16(a1, ahi[ks], bl0, bl1);
-        mma_bf16(a2, alo[ks], bh0, bh1);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x == 1 && !two) break;
+          const int rl = (x ? nt1 : nt0) * 8 + (lane & 7);
+          uint32_t bh0, bh1, bl0, bl1;
+          ldsm_x4(stu + (ks >> 1) * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
+          mma_bf16(a0[x], ahi, bh0, bh1);
+          mma_bf16(a1[x], ahi, bl0, bl1);
+          mma_bf16(a2[x], alo, bh0, bh1);
+        }
       }
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int i = irow[hr];
-        if (i >= Lq) continue;
-        const int cc = cb + nt * 8 + 2 * tq;
-        float z[2];
+      for (int x = 0; x < 2; ++x) {
+        if (x == 1 && !two) break;
+        const int cc = cb + (x ? nt1 : nt0) * 8 + 2 * tq;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = cc + e;
-          const float acc = a0[2 * hr + e] + (a1[2 * hr + e] + a2[2 * hr + e]);
-          z[e] = (c < c1 && chunk_eligible(c, prow[hr], w)) ? tau * acc - lambda * hs[c - c0] : -INFINITY;
-        }
-        float* zr = z_all + ((size_t)(b * Hq + h) * Lq + i) * C;
-        if (cc + 1 < c1 && ((C & 1) == 0)) {
-          *reinterpret_cast<float2*>(zr + cc) = make_float2(z[0], z[1]);
-        } else {
-          if (cc < c1) zr[cc] = z[0];
-          if (cc + 1 < c1) zr[cc + 1] = z[1];
+        for (int hr = 0; hr < 2; ++hr) {
+          const int i = irow[hr];
+          if (i >= Lq) continue;
+          float z[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = cc + e;
+            const float acc = a0[x][2 * hr + e] + (a1[x][2 * hr + e] + a2[x][2 * hr + e]);
+            const bool elig = c < c1 && (c < wlo[hr] || c > whi[hr]);
+            z[e] = elig ? tau * acc - lambda * hs[c - c0] : -INFINITY;
+          }
+          float* zr = z_all + ((size_t)(b * Hq + h) * Lq + i) * C;
+          if (cc + 1 < c1 && ((C & 1) == 0)) {
+            *reinterpret_cast<float2*>(zr + cc) = make_float2(z[0], z[1]);
+          } else {
+            if (cc < c1) zr[cc] = z[0];
+            if (cc + 1 < c1) zr[cc + 1] = z[1];
+          }
         }
       }
     }
-    __syncthreads();                       // stage s consumed by every warp
+    __syncthreads();                       // stage consumed by every warp
     if (tid == 0 && bx + nstg < nb) {
       tc::fence_proxy_async();
-      tc::mbar_arrive_expect_tx(&full[s], (unsigned)boxr * 512u);
-      tc::tma_load_3d(ring + s * boxr * 512, &smap, 0, (int)(srow0 + (size_t)(bx + nstg) * boxr), 0, &full[s]);
+      tc::mbar_arrive_expect_tx(&full[st], (unsigned)boxr * 512u);
+      tc::tma_load_3d(ring + st * boxr * 512, &smap, 0, (int)(srow0 + (size_t)(bx + nstg) * boxr), 0, &full[st]);
     }
   }
   RDL_TRACE_POINT(1, 5);
@@ -447,18 +472,19 @@ constexpr int DK_MAXZ = 8 * 4096;           // floats of staged score rows
 // ranked exactly; more than DK_MAXCAND of them (heavy ties) falls back to the radix select.
 constexpr int DK_MAXCAND = 256;
 
+constexpr int DK_THREADS = 512;
 template <bool ZS, int MAXM>
-__global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__ z_all,
+__global__ void __launch_bounds__(DK_THREADS) dec_topk_kernel(const float* __restrict__ z_all,
                                                        const int32_t* __restrict__ q_pos, int Lq, int L,
                                                        int Hq, int Hkv, int K, int32_t* __restrict__ idx,
                                                        float* __restrict__ z_sel) {
   extern __shared__ __align__(128) uint32_t dk_smem[];
   __shared__ unsigned hist[256];
-  __shared__ unsigned whist[8][256];
-  __shared__ int warp_sums[8];
+  __shared__ unsigned whist[DK_THREADS / 32][256];
+  __shared__ int warp_sums[DK_THREADS / 32];
   __shared__ int sel_s[64];
   __shared__ int bc[3];
-  __shared__ unsigned long long wbound[8];
+  __shared__ unsigned long long wbound[DK_THREADS / 32];
   __shared__ unsigned long long cand[DK_MAXCAND];
   __shared__ int ncand_s;
   __shared__ __align__(8) uint64_t zbar;
@@ -481,7 +507,7 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__
   const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
   int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
   if (is_mask_slot(p)) {
-    for (int e = tid; e < K * G; e += 256) {
+    for (int e = tid; e < K * G; e += DK_THREADS) {
       const int k = e % K, hl = e / K;
       if (hl == 0) irow[k] = -1;
       z_sel[((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k] = -INFINITY;
@@ -497,13 +523,13 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__
     (void)tc::mbar_wait(&zbar, 0);
   }
   const uint32_t kneg = order_key(-INFINITY);
-  // thread t owns chunks t + 256 m (m < MAXM, C <= 256 MAXM); packed keys stay in registers
-  const int nm = (C + 255) / 256;
+  // thread t owns chunks t + 512 m (m < MAXM, C <= 512 MAXM); packed keys stay in registers
+  const int nm = (C + DK_THREADS - 1) / DK_THREADS;
   unsigned long long pk[MAXM];
 #pragma unroll
   for (int m = 0; m < MAXM; ++m) {
     pk[m] = 0ull;
-    const int c = tid + 256 * m;
+    const int c = tid + DK_THREADS * m;
     if (m < nm && c < C) {
       float zz;
       if (ZS) {
@@ -520,7 +546,8 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__
   }
   RDL_TRACE_POINT(2, 2);
   // per-warp q-th largest packed key (0 when the warp has fewer than q valid keys)
-  const int qk = (K + 7) / 8;
+  constexpr int NW = DK_THREADS / 32;
+  const int qk = (K + NW - 1) / NW;
   {
     unsigned long long last = ~0ull, bound = 0ull;
     for (int r = 0; r < qk; ++r) {
@@ -543,7 +570,7 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__
   __syncthreads();
   unsigned long long L0 = wbound[0];
 #pragma unroll
-  for (int w8 = 1; w8 < 8; ++w8) L0 = wbound[w8] < L0 ? wbound[w8] : L0;
+  for (int w8 = 1; w8 < NW; ++w8) L0 = wbound[w8] < L0 ? wbound[w8] : L0;
   if (L0 == 0ull) L0 = 1ull;      // fewer than K valid keys in some warp: every valid key is a candidate
   // candidates: keys >= L0
 #pragma unroll
@@ -576,11 +603,13 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const float* __restrict__
     if (tid < nsel) sel_s[pos] = c_mine;
     __syncthreads();
   } else {
+    // heavy ties: the radix select over all keys (written for 256 threads; the other
+    // threads take part in its barriers only)
     __syncthreads();
-    nsel = cta_select_topk(keys, C, K, hist, whist, warp_sums, bc, sel_s);
+    nsel = cta_select_topk_t<DK_THREADS>(keys, C, K, hist, whist, warp_sums, bc, sel_s);
   }
   RDL_TRACE_POINT(2, 3);
-  for (int e = tid; e < K * G; e += 256) {
+  for (int e = tid; e < K * G; e += DK_THREADS) {
     const int k = e % K, hl = e / K;
     const int c = k < nsel ? sel_s[k] : -1;
     if (hl == 0) irow[k] = c;
@@ -726,7 +755,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   }
   for (int e = tid; e < Lq; e += AT_THREADS) pos_s[e] = q_pos ? q_pos[(size_t)b * Lq + e] : e;
-  for (int e = tid; e < Lq * 8 * 16; e += AT_THREADS) {
+  cp_async_commit();                      // group 1: idx; group 2: the query rows (waited for later)
+  for (int e = tid; e < Lq * 8 * 16 && tid < AT_CONS * 32; e += AT_CONS * 32) {   // consumer threads only
     const int i = e >> 7, hd = (e >> 4) & 7, u = e & 15;
     unsigned char* dst = qs + i * 2048 + hd * 256 + ((u ^ hd) << 4);
     if (hd < G)
@@ -736,7 +766,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   }
   cp_async_commit();
   for (int c = tid; c < C; c += AT_THREADS) hist[c] = 0;
-  cp_async_wait<0>();
+  cp_async_wait<1>();
   __syncthreads();
   RDL_TRACE_POINT(3, 4);
   // ---------------- tasks per slab (the same on every CTA of the group)
@@ -792,49 +822,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   }
   RDL_TRACE_POINT(3, 6);
-  // task cursors: pre[c] = first list position of slab c (prefix of the task counts)
-  {
-    int local = 0;
-    for (int c = s0; c < s1; ++c) local += hist[c];
-    int total;
-    int run = cta_excl_scan(local, scan_ws, total);
-    for (int c = s0; c < s1; ++c) {
-      pre[c] = run;
-      run += hist[c];
-    }
-  }
   __syncthreads();
   const int c_lo = misc[0], c_hi = misc[1] + 1;     // empty when c_lo > c_hi - 1
-  const int lbase = c_lo < c_hi ? pre[c_lo] : 0;   // list positions relative to this CTA
-  const int lcap = Lq * (Kt + nwt);
-  __syncthreads();
-  if (ROUTE && c_lo < c_hi) {
-    for (int e = tid; e < nent; e += AT_THREADS) {
-      const int c = idx_s[e];
-      if (c < c_lo || c >= c_hi || !chunk_ok(e, c)) continue;
-      const int slot = atomicAdd(&pre[c], 1) - lbase;
-      if (slot < lcap) list[slot] = ((e / K) << 8) | (e % K);
-      else record_status(RDL_ERR_DEVICE_CHECK);
-    }
-  }
-  if (w >= 0 && c_lo < c_hi) {
-    for (int i = warp; i < Lq; i += AT_CONS + 1) {
-      const int p = pos_s[i];
-      if (ROUTE && is_mask_slot(p)) continue;
-      const int lo = win_lo(p, w), hi = min(win_hi(p, w, L), c_hi - 1);
-      for (int t = max(lo, c_lo) + lane; t <= hi; t += 32) {
-        const int slot = atomicAdd(&pre[t], 1) - lbase;
-        if (slot < lcap) list[slot] = (i << 8) | TASK_WIN | (t - lo);
-        else record_status(RDL_ERR_DEVICE_CHECK);
-      }
-    }
-  }
-  __syncthreads();
-  RDL_TRACE_POINT(3, 2);
-  // after the scatter pre[c] = end of slab c's tasks (absolute); start = end - hist[c]
 
   if (warp == AT_CONS) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer: starts while the consumers build the task lists
     if (lane == 0) {
       int u = 0;
       int last_issued[4] = {-1, -1, -1, -1};
@@ -861,7 +853,61 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     return;
   }
 
-  // ---------------- consumer warps: pairs of tasks, pair index % 8 == warp
+  // ---------------- consumer warps only from here (named barrier 1, AT_CONS warps)
+  // task cursors: pre[c] = first list position of slab c (prefix of the task counts)
+  {
+    constexpr int NCT = AT_CONS * 32;
+    const int cseg = (C + NCT - 1) / NCT;
+    const int q0 = min(C, tid * cseg), q1 = min(C, q0 + cseg);
+    int local = 0;
+    for (int c = q0; c < q1; ++c) local += hist[c];
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scan_ws[warp] = x;
+    asm volatile("bar.sync 1, %0;\n" ::"n"(NCT) : "memory");
+    int run = 0;
+    for (int w8 = 0; w8 < warp; ++w8) run += scan_ws[w8];
+    run += x - local;
+    for (int c = q0; c < q1; ++c) {
+      pre[c] = run;
+      run += hist[c];
+    }
+    asm volatile("bar.sync 1, %0;\n" ::"n"(NCT) : "memory");
+  }
+  const int lbase = c_lo < c_hi ? pre[c_lo] : 0;   // list positions relative to this CTA
+  const int lcap = Lq * (Kt + nwt);
+  asm volatile("bar.sync 1, %0;\n" ::"n"(AT_CONS * 32) : "memory");
+  if (ROUTE && c_lo < c_hi) {
+    for (int e = tid; e < nent; e += AT_CONS * 32) {
+      const int c = idx_s[e];
+      if (c < c_lo || c >= c_hi || !chunk_ok(e, c)) continue;
+      const int slot = atomicAdd(&pre[c], 1) - lbase;
+      if (slot < lcap) list[slot] = ((e / K) << 8) | (e % K);
+      else record_status(RDL_ERR_DEVICE_CHECK);
+    }
+  }
+  if (w >= 0 && c_lo < c_hi) {
+    for (int i = warp; i < Lq; i += AT_CONS) {
+      const int p = pos_s[i];
+      if (ROUTE && is_mask_slot(p)) continue;
+      const int lo = win_lo(p, w), hi = min(win_hi(p, w, L), c_hi - 1);
+      for (int t = max(lo, c_lo) + lane; t <= hi; t += 32) {
+        const int slot = atomicAdd(&pre[t], 1) - lbase;
+        if (slot < lcap) list[slot] = (i << 8) | TASK_WIN | (t - lo);
+        else record_status(RDL_ERR_DEVICE_CHECK);
+      }
+    }
+  }
+  RDL_TRACE_POINT(3, 2);
+  // after the scatter pre[c] = end of slab c's tasks (absolute); start = end - hist[c]
+
+  // ---------------- consumer warps: pairs of tasks, pair index % AT_CONS == warp
+  cp_async_wait<0>();
+  asm volatile("bar.sync 1, %0;\n" ::"n"(AT_CONS * 32) : "memory");   // query rows visible to every consumer
   int u = 0, pair0 = 0;
   for (int c = c_lo; c < c_hi; ++c) {
     const int n = hist[c];

@@ -443,18 +443,46 @@ __device__ __forceinline__ int block_excl_scan256(int v, int* warp_sums, int& to
   return base + x - v;
 }
 
-// Exact top-K of the order keys keys[0..C) by one CTA of 256 threads: a 4-pass 8-bit radix
-// select for the K-th largest key, then an in-order compaction that takes every key above it
-// and the first (by chunk index) of the keys equal to it.  sel_s receives the selected
-// chunk indices in ascending order; returns how many there are (min(#valid, K)).
-__device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int K, unsigned* hist,
-                                               unsigned (*whist)[256], int* warp_sums, int* bc, int* sel_s) {
+// Block-wide exclusive scan of one int per thread (NT threads); returns the total.
+template <int NT>
+__device__ __forceinline__ int block_excl_scan_t(int v, int* warp_sums, int& total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < NW; ++w8) {
+    const int ws = warp_sums[w8];
+    if (w8 < warp) base += ws;
+    tot += ws;
+  }
+  __syncthreads();
+  total = tot;
+  return base + x - v;
+}
+
+// Exact top-K of the order keys keys[0..C) by one CTA of NT threads (NT >= 256): a 4-pass
+// 8-bit radix select for the K-th largest key, then an in-order compaction that takes every
+// key above it and the first (by chunk index) of the keys equal to it.  sel_s receives the
+// selected chunk indices in ascending order; returns how many there are (min(#valid, K)).
+// whist: NT/32 per-warp histograms of 256 bins; warp_sums: NT/32 ints.
+template <int NT>
+__device__ __forceinline__ int cta_select_topk_t(const uint32_t* keys, int C, int K, unsigned* hist,
+                                                 unsigned (*whist)[256], int* warp_sums, int* bc, int* sel_s) {
+  constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t kneg = order_key(-INFINITY);
   int nv = 0;
-  for (int c = tid; c < C; c += 256) nv += keys[c] > kneg;
+  for (int c = tid; c < C; c += NT) nv += keys[c] > kneg;
   int nvalid;
-  (void)block_excl_scan256(nv, warp_sums, nvalid);
+  (void)block_excl_scan_t<NT>(nv, warp_sums, nvalid);
   uint32_t thr = kneg;
   int need = 0;
   if (nvalid > K) {
@@ -466,17 +494,17 @@ __device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int 
 #pragma unroll
       for (int u = 0; u < 8; ++u) whist[warp][lane * 8 + u] = 0;
       __syncwarp();
-      for (int base = 0; base < C; base += 256) {
+      for (int base = 0; base < C; base += NT) {
         const int c = base + tid;
         const uint32_t k = c < C ? keys[c] : 0u;
         if (c < C && (k & pmask) == prefix) atomicAdd(&whist[warp][(k >> shift) & 255u], 1u);
       }
       __syncwarp();
       __syncthreads();
-      {
+      if (tid < 256) {
         unsigned sum = 0;
 #pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) sum += whist[w8][tid];
+        for (int w8 = 0; w8 < NW; ++w8) sum += whist[w8][tid];
         hist[tid] = sum;
       }
       __syncthreads();
@@ -516,7 +544,7 @@ __device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int 
     thr = prefix;
   }
   // ordered compaction: thread t owns the contiguous range [t*seg, (t+1)*seg)
-  const int seg = (C + 255) / 256, c0 = tid * seg, c1 = min(C, c0 + seg);
+  const int seg = (C + NT - 1) / NT, c0 = tid * seg, c1 = min(C, c0 + seg);
   int ngt = 0, nties = 0;
   for (int c = c0; c < c1; ++c) {
     const uint32_t k = keys[c];
@@ -524,9 +552,9 @@ __device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int 
     nties += (need > 0 && k == thr);
   }
   int tot;
-  const int tie_base = block_excl_scan256(nties, warp_sums, tot);
+  const int tie_base = block_excl_scan_t<NT>(nties, warp_sums, tot);
   const int take_ties = max(0, min(nties, need - tie_base));
-  const int pos0 = block_excl_scan256(ngt + take_ties, warp_sums, tot);
+  const int pos0 = block_excl_scan_t<NT>(ngt + take_ties, warp_sums, tot);
   int pos = pos0, tk = 0;
   for (int c = c0; c < c1; ++c) {
     const uint32_t k = keys[c];
@@ -537,6 +565,10 @@ __device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int 
   }
   __syncthreads();
   return min(tot, K);
+}
+__device__ __forceinline__ int cta_select_topk(const uint32_t* keys, int C, int K, unsigned* hist,
+                                               unsigned (*whist)[256], int* warp_sums, int* bc, int* sel_s) {
+  return cta_select_topk_t<256>(keys, C, K, hist, whist, warp_sums, bc, sel_s);
 }
 
 // One CTA (256 threads) per (b, g, i): the same exact top-K as topk_radix_kernel, for few
