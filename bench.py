@@ -214,6 +214,7 @@ def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
     from diffusion_lms_b200 import workloads as W
     wd = W.decode_128k(seed=rank_seed(3, rank))
     dinp = api.to_device(wd, dev)
+    dinp.dims.flags = rdl.FLAG_SPLIT_SUMMARY      # summaries pooled once per block, pre-split
     dout = api.alloc_outputs(dinp.dims, dinp.dtype, dev)
     api.summary_pool(dinp, dout, stream=stream)
 

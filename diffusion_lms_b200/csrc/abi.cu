@@ -299,8 +299,11 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
   const int C = dm->L / S, M = dm->B * dm->Lq;
   const bool res = dm->r > 0 && x;
   const DecScoreGrid gr = dec_score_grid(dm);
+  const bool split = (dm->flags & RDL_FLAG_SPLIT_SUMMARY) != 0;
   CUtensorMap smap;
-  if (!make_tmap_f32_rows(&smap, summary, (unsigned long long)dm->B * dm->Hq * C, (unsigned)gr.boxr))
+  const unsigned long long srows = (unsigned long long)dm->B * dm->Hq * C;
+  if (split ? !make_tmap_split_rows(&smap, summary, srows, (unsigned)gr.boxr)
+            : !make_tmap_f32_rows(&smap, summary, srows, (unsigned)gr.boxr))
     return RDL_ERR_CUDA;
   if (res) {
     const int slice = ((dm->D + dec::TK_CL * 64 - 1) / (dec::TK_CL * 64)) * 64;
@@ -317,7 +320,10 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
         cudaSuccess)
       return RDL_ERR_CUDA;
   }
-  auto kern = gr.MT == 1 ? dec::dec_score_kernel<1> : (gr.MT == 2 ? dec::dec_score_kernel<2> : dec::dec_score_kernel<4>);
+  auto kern = split ? (gr.MT == 1 ? dec::dec_score_kernel<1, true>
+                                  : (gr.MT == 2 ? dec::dec_score_kernel<2, true> : dec::dec_score_kernel<4, true>))
+                    : (gr.MT == 1 ? dec::dec_score_kernel<1, false>
+                                  : (gr.MT == 2 ? dec::dec_score_kernel<2, false> : dec::dec_score_kernel<4, false>));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gr.smem) != cudaSuccess)
     return RDL_ERR_CUDA;
   const float tau = (float)(1.0 / sqrt((double)dm->d));
@@ -634,6 +640,7 @@ rdl_status rdl_route_score_topk(const void* q, const int32_t* q_pos, const void*
   const cudaStream_t st = as_stream(stream);
   if (dec_score_ok(&dm, dtype))
     return score_decode(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel, workspace, st);
+  if (dm.flags & RDL_FLAG_SPLIT_SUMMARY) return RDL_ERR_UNSUPPORTED;
   if (fast_score(&dm, dtype))
     return score_fast(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx, z_sel, workspace, st);
   return dtype == RDL_BF16 ? score_impl<__nv_bfloat16>(q, q_pos, x, w_down, w_up, summary, entropy, &dm, idx,

@@ -211,7 +211,7 @@ __host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nst
 // byte offset of 16-byte unit u (0..31: hi 0-15, lo 16-31) of row `row` in a qsp tile
 __device__ __forceinline__ uint32_t qsp_off(int row, int u) { return (uint32_t)(row * 512 + ((u ^ (row & 7)) << 4)); }
 
-template <int MT>
+template <int MT, bool SPLIT>
 __global__ void __launch_bounds__(SC_WARPS * 32, 1)
     dec_score_kernel(const __grid_constant__ CUtensorMap smap, const float* __restrict__ smap_base,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
@@ -358,8 +358,8 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
       whi[hr] = (p + w) / S;
     }
   }
-  // ---- scores over the range, box by box as the TMA loads land.  Each landed box is first
-  // rewritten in place: every 128-byte segment (32 fp32 of one summary row) becomes 32 bf16
+  // ---- scores over the range, box by box as the TMA loads land.  An fp32 box is first
+  // rewritten in place (a box of split-layout summaries is used as it lands): every 128-byte segment (32 fp32 of one summary row) becomes 32 bf16
   // hi terms (logical 16-byte units 0-3) and 32 bf16 lo terms (units 4-7), x = hi + lo to
   // ~2^-17, keeping the unit ^ (row % 8) swizzle so the fragment loads stay conflict-free.
   const int ntb = boxr / 8;
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
     if (bx == 1) RDL_TRACE_POINT(1, 6);
     if (bx == nb - 1) RDL_TRACE_POINT(1, 7);
     unsigned char* stg = ring + st * boxr * 512;
-    for (int seg = tid; seg < 4 * boxr; seg += NT) {
+    for (int seg = tid; !SPLIT && seg < 4 * boxr; seg += NT) {
       const int rr = seg % boxr;
       unsigned char* sp = stg + (seg / boxr) * boxr * 128 + rr * 128;
       const int sw = rr & 7;
@@ -409,13 +409,16 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
         const int ra = mw * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), ua = 2 * ks + (lane >> 4);
         ldsm_x4(smem_u32(qsp + qsp_off(ra, ua)), ahi[0], ahi[1], ahi[2], ahi[3]);
         ldsm_x4(smem_u32(qsp + qsp_off(ra, 16 + ua)), alo[0], alo[1], alo[2], alo[3]);
-        const int un = (mj >= 2 ? 4 : 0) + ((16 * ks) & 31) / 8 + (mj & 1);
+        // converted fp32 box: slice ks/2, units hi 0-3 / lo 4-7; split-layout box: segments
+        // hi (ks/4), lo (2 + ks/4), units 2 (ks % 4) + {0, 1}
+        const int un = SPLIT ? 2 * (ks & 3) + (mj & 1) : (mj >= 2 ? 4 : 0) + ((16 * ks) & 31) / 8 + (mj & 1);
+        const int sg = SPLIT ? (mj >= 2 ? 2 : 0) + (ks >> 2) : (ks >> 1);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           if (x == 1 && !two) break;
           const int rl = (x ? nt1 : nt0) * 8 + (lane & 7);
           uint32_t bh0, bh1, bl0, bl1;
-          ldsm_x4(stu + (ks >> 1) * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
+          ldsm_x4(stu + sg * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
           mma_bf16(a0[x], ahi, bh0, bh1);
           mma_bf16(a1[x], ahi, bl0, bl1);
           mma_bf16(a2[x], alo, bh0, bh1);

@@ -91,8 +91,19 @@ __global__ void __launch_bounds__(256) summary_pool_kernel(
       }
     }
     float* srow = summary + ((size_t)(b * Hq + h) * C + c) * D;
+    if (flags & RDL_FLAG_SPLIT_SUMMARY) {
+      // the same 4D bytes as D bf16 hi terms, then D bf16 lo terms (s = hi + lo)
+      __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(srow);
 #pragma unroll
-    for (int u = 0; u < EPL; ++u) srow[lane + 32 * u] = sacc[u];
+      for (int u = 0; u < EPL; ++u) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(sacc[u]);
+        hrow[lane + 32 * u] = hi;
+        hrow[D + lane + 32 * u] = __float2bfloat16_rn(sacc[u] - __bfloat162float(hi));
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < EPL; ++u) srow[lane + 32 * u] = sacc[u];
+    }
     if (lane == 0) entropy[(size_t)(b * Hq + h) * C + c] = H;
     if (o_mask && v) {
       T* orow = o_mask + (size_t)b * q_batch_stride + (size_t)c * q_chunk_stride + (size_t)h * D;

@@ -88,4 +88,19 @@ inline bool make_tmap_f32_rows(CUtensorMap* map, const void* base, unsigned long
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Summaries in the split layout ([hi 128 | lo 128] bf16, 512 B per row) viewed as
+// (64 columns, rows, 4 segments): one box of box_rows rows lands as 4 segments [box_rows][128 B]
+// (hi 0-63, hi 64-127, lo 0-63, lo 64-127), each with the 128-byte swizzle.
+inline bool make_tmap_split_rows(CUtensorMap* map, const void* base, unsigned long long rows, unsigned box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, 4};
+  cuuint64_t strides[2] = {512, 128};
+  cuuint32_t box[3] = {64, box_rows, 4};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace rdl

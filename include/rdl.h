@@ -18,7 +18,8 @@
  *   x          [B, Lq, D]       storage dtype;   w_down [D, r];  w_up [r, Hq*d]
  *   q_pos      [B, Lq] int32    position of each query row; NULL means row i is at
  *                               position i (then Lq must equal L)
- *   summary    [B, Hq, C, d]    fp32;            entropy [B, Hq, C] fp32
+ *   summary    [B, Hq, C, d]    fp32 (or the split layout of RDL_FLAG_SPLIT_SUMMARY);
+ *                               entropy [B, Hq, C] fp32
  *   idx        [B, Hkv, Lq, K]  int32: selected chunks in ascending order, then -1
  *   z_sel      [B, Hq, Lq, K]   fp32: route score of each selected chunk for each head
  *                               (-inf in padded slots)
@@ -65,6 +66,13 @@ typedef enum { RDL_BF16 = 0, RDL_F32 = 1 } rdl_dtype;
 /* flags */
 #define RDL_FLAG_MEAN_SUMMARY 0x1 /* summary = mean of the 63 content keys (Table 6 ablation) */
 #define RDL_FLAG_CHECKS 0x2       /* device-side index/position checks into the status word */
+/* Summary layout for decode blocks: rdl_summary_pool writes, and rdl_route_score_topk reads,
+ * each summary row as d bf16 "hi" terms followed by d bf16 "lo" terms (s = hi + lo to about
+ * 2^-17 relative; the same 4d bytes as the fp32 row).  The split is then done once when the
+ * block's summaries are pooled instead of on every decode step.  rdl_route_score_topk accepts
+ * it for decode-block shapes (bf16, d = 128, at most 64 rows) and returns
+ * RDL_ERR_UNSUPPORTED otherwise. */
+#define RDL_FLAG_SPLIT_SUMMARY 0x4
 
 #define RDL_CHUNK 64
 

@@ -52,7 +52,11 @@ def run_gpu(wl: Workload, *, flags=0, with_residual=True, route=True, swa=False)
     torch.cuda.synchronize()
     st = rdl.rdl_last_device_status()
     assert st == rdl.OK, rdl.status_string(st)
-    res.update(s=out.s.double().cpu().numpy(), H=out.H.double().cpu().numpy(),
+    s_out = out.s
+    if flags & rdl.FLAG_SPLIT_SUMMARY:     # rows of [hi d | lo d] bf16: s = hi + lo
+        sp = out.s.view(torch.bfloat16).reshape(*out.s.shape[:-1], 2, out.s.shape[-1])
+        s_out = sp[..., 0, :].double() + sp[..., 1, :].double()
+    res.update(s=s_out.double().cpu().numpy(), H=out.H.double().cpu().numpy(),
                idx=out.idx.cpu().numpy().astype(np.int64), z=out.z_sel.double().cpu().numpy(),
                o=out.o.double().cpu().numpy(), lse=out.lse.double().cpu().numpy())
     if swa:

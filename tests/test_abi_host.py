@@ -117,3 +117,10 @@ def test_raise_on_error():
 
 def test_dims_struct_layout():
     assert ctypes.sizeof(rdl.rdl_dims) == 12 * 4
+
+
+def test_split_summary_layout_only_on_decode_blocks():
+    """The split summary layout is read by the decode-block scorer only; other shapes refuse
+    it before launching anything."""
+    dm = dims(flags=rdl.FLAG_SPLIT_SUMMARY)          # fp32, d = 64, prefill-shaped
+    assert _score(dm) == rdl.ERR_UNSUPPORTED

@@ -43,10 +43,13 @@ def test_bf16_prefill_ragged_every_row():
     P.check_swa(wl, gpu, rows)
 
 
-def test_bf16_decode_block_split_path():
+@pytest.mark.parametrize("split", [False, True])
+def test_bf16_decode_block(split):
+    """32-query decode block; with the split summary layout the pooled summaries are stored
+    as bf16 hi/lo rows and the scorer reads them directly."""
     dm = small(L=8192, Lq=32, K=32, w=256)
     wl = W.make_inputs(dm, seed=12, n_needles=8, decode_block=32)
-    gpu = P.run_gpu(wl, swa=True)
+    gpu = P.run_gpu(wl, swa=True, flags=rdl.FLAG_SPLIT_SUMMARY if split else 0)
     rows = np.arange(32)
     P.check_route_layer(wl, gpu, rows)
     P.check_swa(wl, gpu, rows)
