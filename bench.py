@@ -5,7 +5,8 @@ rdl_route_score_topk + rdl_route_attn on the 16K Dream-7B-shaped prefill (28 que
 4 KV heads, head dim 128, K = 32 chunks, window radius 256, rank-64 residual), inputs
 resident in HBM.  The metric is route-layer query tokens per second (content rows; the
 mask-slot rows are produced by the summary pool inside the same step).  The JSON line
-also carries the 128K decode block (score + attention with cached summaries, ms per step).
+also carries the 128K decode block (score + attention with cached summaries, ms per step)
+and the 28-layer 128K attention stack (ms per denoising step).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -272,6 +273,88 @@ def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
                          "peak_source": f"hbm_gbs ({pk_kind})"}}
 
 
+def stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind):
+    """28-layer attention stack at 128K for one 32-query decode block (every 4th layer a
+    route layer: score + two-level attention over cached pre-split summaries; the other 21
+    the bidirectional sliding window), all 28 layers captured in one CUDA graph and replayed;
+    L2 flushed between replays (untimed).  Inputs are drawn on the device (N(0,1) K/V/Q/x,
+    N(0, 0.02^2) residual weights), the shapes of the 28-layer stack workload."""
+    import torch
+    from diffusion_lms_b200 import api, rdl
+    from diffusion_lms_b200.workloads import STACK_LAYERS, is_route_layer
+    L, Lq, Hq, Hkv, d, D, r, K, w = 131072, 32, 28, 4, 128, 3584, 64, 32, 256
+    C = L // 64
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(rank_seed(5, rank))
+
+    def rn(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=gen, device=dev) * scale).to(torch.bfloat16)
+
+    q_pos = torch.arange(L - 64, L - 32, dtype=torch.int32, device=dev)[None]
+    layers = []
+    for layer in range(STACK_LAYERS):
+        route = is_route_layer(layer)
+        dm = rdl.Dims(B=1, L=L, Lq=Lq, Hq=Hq, Hkv=Hkv, d=d, D=D, r=r, K=K, w=w, lam=0.1,
+                      flags=rdl.FLAG_SPLIT_SUMMARY if route else 0)
+        inp = api.DeviceInputs(dm, "bf16", rn(1, Lq, Hq, d), rn(1, Hkv, L, d), rn(1, Hkv, L, d),
+                               rn(1, Lq, D), rn(D, r, scale=0.02), rn(r, Hq * d, scale=0.02),
+                               q_pos, rn(1, C, Hq, d) if route else None)
+        out = api.alloc_outputs(dm, "bf16", dev)
+        if route:
+            api.summary_pool(inp, out, stream=stream)     # once per block, untimed
+        layers.append((route, inp, out))
+    torch.cuda.synchronize()
+
+    def run(st):
+        for route, inp, out in layers:
+            if route:
+                api.score_topk(inp, out, stream=st)
+                api.route_attn(inp, out, stream=st)
+            else:
+                api.swa_attn(inp, out, stream=st)
+
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        run(cs)
+    torch.cuda.synchronize()
+    launches0 = rdl.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            run(cs)
+    launches = rdl.launch_count() - launches0
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s_ in range(args.steps):
+        flush.zero_()
+        ev[s_][0].record(stream)
+        g.replay()
+        ev[s_][1].record(stream)
+    torch.cuda.synchronize()
+    ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+    assert rdl.rdl_last_device_status() == rdl.OK
+    # bytes the step must move: per route layer as decode_bytes, per window layer its K/V
+    # window plus queries and outputs
+    by = 0
+    for route, inp, out in layers:
+        if route:
+            by += decode_bytes(inp.dims, out.idx.cpu().numpy())["total"]
+        else:
+            by += min(L, 64 + 2 * w) * Hkv * 2 * d * 2 + 2 * Lq * 2 * Hq * d
+    ach = by / (ms / 1e3) / 1e9
+    del g
+    return {"workload": "stack_128k (28 layers: 7 route, 21 sliding window)", "ms_per_step": ms,
+            "timing": "one CUDA graph of all 28 layers, median of replays, L2 flushed between",
+            "kernels_per_step": launches,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "algorithmic_bytes": by,
+                         "peak_source": f"hbm_gbs ({pk_kind})"}}
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def main():
@@ -283,6 +366,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=96)
     ap.add_argument("--cpu-rows", type=int, default=96)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--stack-only", action="store_true",
+                    help="time only the 28-layer 128K stack (profiling aid)")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the 128K decode block (profiling aid)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -320,6 +406,11 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
     pk, pk_kind = peaks()
+    if args.stack_only:
+        st_ = stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"stack_128k": st_}), flush=True)
+        return
     if args.decode_only:
         dec = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
         if rank == 0:
@@ -430,6 +521,10 @@ def main():
         del inp, out
         torch.cuda.empty_cache()
         decode = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
+    stack = None
+    if not args.no_stack:
+        torch.cuda.empty_cache()
+        stack = stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind)
 
     # ---------------- CPU baseline (rank 0, oracle on a bounded sample)
     cpu = None
@@ -449,7 +544,7 @@ def main():
                            "l2": "flushed between timed steps (256 MB write, untimed)",
                            "parallelism": f"independent sequence per GPU x{world}"},
                 "breakdown_ms": calls, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk, "decode_128k": decode}
+                "gpu_launches": launches, "clocks": clk, "decode_128k": decode, "stack_128k": stack}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -241,11 +241,7 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
 // Sliding-window workspace: key-split partials when the row count is small (else none).
 size_t swa_ws(const rdl_dims* dm, rdl_dtype t) {
   if (!fast_attn(dm, t) || dm->w < 0) return 0;
-  if (dec_swa_ok(dm, t) && dec_attn_stages(dm, 0) > 0) {
-    const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
-    const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
-    return align256(sizeof(float) * rows * nwt * dm->d) + align256(sizeof(float2) * rows * nwt);
-  }
+  if (dec_swa_ok(dm, t)) return 0;
   const int nsw = window_splits(dm);
   if (nsw <= 1) return 0;
   const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
@@ -374,36 +370,6 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
   if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, st, q_pos, idx, z_sel,
                  (const float*)o_part, (const float*)ow_part, (const float2*)ml_part, dm->B, dm->L, dm->Lq, dm->Hq,
                  dm->Hkv, dm->K, dm->w, dm->flags, static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
-    return RDL_ERR_CUDA;
-  return RDL_OK;
-}
-
-rdl_status swa_decode(const void* q, const int32_t* q_pos, const void* k, const void* v, const rdl_dims* dm, void* o,
-                      float* lse, void* workspace, cudaStream_t st) {
-  const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
-  const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
-  float* ow_part = static_cast<float*>(workspace);
-  float2* ml_part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + align256(sizeof(float) * rows * nwt * dm->d));
-  const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
-  CUtensorMap kmap, vmap;
-  if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
-  const int stages = dec_attn_stages(dm, 0);
-  const int smem = dec::attn_smem(stages, dm->Lq, 0, dm->L / S, (int)nwt).total;
-  auto kern = dec::dec_attn_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return RDL_ERR_CUDA;
-  const float sl2 = (float)(1.0 / sqrt((double)dm->d) * 1.4426950408889634);
-  const int R = dec_attn_ranges(dm);
-  if (launch_pdl(kern, dim3(dm->B * dm->Hkv * R), dim3(dec::AT_THREADS), smem, st, kmap, vmap,
-                 static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-                 static_cast<const __nv_bfloat16*>(q), q_pos, (const int32_t*)nullptr, dm->L, dm->Lq, dm->Hq,
-                 dm->Hkv, 0, dm->w, dm->flags, R, stages, sl2, (float*)nullptr, ow_part, ml_part) != cudaSuccess)
-    return RDL_ERR_CUDA;
-  const long long items = (long long)dm->B * dm->Lq * dm->Hq;
-  if (launch_pdl(dec::dec_comb_kernel<false>, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, st, q_pos,
-                 (const int32_t*)nullptr, (const float*)nullptr, (const float*)nullptr, (const float*)ow_part,
-                 (const float2*)ml_part, dm->B, dm->L, dm->Lq, dm->Hq, dm->Hkv, 0, dm->w, dm->flags,
-                 static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
     return RDL_ERR_CUDA;
   return RDL_OK;
 }
@@ -739,10 +705,21 @@ rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, cons
                              : generic_attn<float, false>(q, q_pos, k, v, nullptr, nullptr, dims, o, lse, st);
   }
   const size_t need = swa_ws(dims, dtype);
-  if (dec_swa_ok(dims, dtype) && dec_attn_stages(dims, 0) > 0 && workspace) {
-    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RDL_ERR_INVALID_ARG;
-    if (ws_bytes < need) return RDL_ERR_WORKSPACE;
-    return swa_decode(q, q_pos, k, v, dims, o, lse, workspace, st);
+  if (dec_swa_ok(dims, dtype)) {
+    // decode blocks: one launch, one CTA per (b, group, pair of rows); no workspace
+    const unsigned long long kvrows = (unsigned long long)dims->B * dims->Hkv * dims->L;
+    CUtensorMap kmap, vmap;
+    if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
+    const int smem = dec::swa_smem();
+    if (cudaFuncSetAttribute(dec::dec_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    const float sl2 = (float)(1.0 / sqrt((double)dims->d) * 1.4426950408889634);
+    const int ctas = dims->B * dims->Hkv * ((dims->Lq + 1) / 2);
+    if (launch_pdl(dec::dec_swa_kernel, dim3(ctas), dim3(dec::SW_WARPS * 32), smem, st, kmap, vmap,
+                   static_cast<const __nv_bfloat16*>(q), q_pos, dims->L, dims->Lq, dims->Hq, dims->Hkv, dims->w, sl2,
+                   static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    return RDL_OK;
   }
   if (need == 0 || !workspace) return launch_window_mma<0>(q, q_pos, k, v, dims, o, lse, nullptr, nullptr, 1, st);
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RDL_ERR_INVALID_ARG;

@@ -1054,6 +1054,229 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 }
 
 // =====================================================================================
+// dec_swa_kernel: bidirectional sliding window for decode blocks, one launch.
+// CTA = (b, g, pair of query rows); warp w streams window slabs w, w + SW_WARPS, ... of the
+// pair through its own shared-memory slot (TMA), keeps an online softmax per row (M = 16 =
+// two rows x 8 head slots), and the warps' partial states are merged in a fixed order.
+// =====================================================================================
+constexpr int SW_WARPS = 6;
+
+__host__ __device__ inline int swa_smem() { return 1024 + SW_WARPS * AT_STAGE_BYTES + 2 * 2048 + 64 * SW_WARPS; }
+
+__global__ void __launch_bounds__(SW_WARPS * 32, 1)
+    dec_swa_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                   const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos, int L, int Lq, int Hq,
+                   int Hkv, int w, float sl2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  constexpr int D = 128;
+  extern __shared__ unsigned char sw_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sw_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* slabs = base;                                   // [SW_WARPS][32 KB]
+  unsigned char* qs = slabs + SW_WARPS * AT_STAGE_BYTES;         // [2 rows][8 heads][256 B]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(qs + 2 * 2048);    // one per warp
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int npair = (Lq + 1) / 2;
+  const int pr = blockIdx.x % npair, g = (blockIdx.x / npair) % Hkv, b = blockIdx.x / (npair * Hkv);
+  const int iA = 2 * pr, iB = min(2 * pr + 1, Lq - 1);
+  const bool hasB = 2 * pr + 1 < Lq;
+  if (tid == 0) {
+    for (int x = 0; x < SW_WARPS; ++x) tc::mbar_init(&bar[x], 1);
+    tc::mbar_fence_init();
+  }
+  grid_dep_wait();
+  grid_dep_launch();
+  const int pA = q_pos ? q_pos[(size_t)b * Lq + iA] : iA;
+  const int pB = q_pos ? q_pos[(size_t)b * Lq + iB] : iB;
+  // query rows of the pair: [row][8 heads][256 B], 16-byte units ^ head; head 7+ zero
+  for (int e = tid; e < 2 * 8 * 16; e += SW_WARPS * 32) {
+    const int r = e >> 7, hd = (e >> 4) & 7, u = e & 15;
+    unsigned char* dst = qs + r * 2048 + hd * 256 + ((u ^ hd) << 4);
+    if (hd < G)
+      cp_async16(smem_u32(dst), q + ((size_t)(b * Lq + (r ? iB : iA)) * Hq + g * G + hd) * D + u * 8);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
+  // slabs of the two windows: [loA, hiA] and [loB, hiB] (the union, in order)
+  int loA = win_lo(pA, w), hiA = win_hi(pA, w, L), loB = win_lo(pB, w), hiB = win_hi(pB, w, L);
+  if (loB < loA) {
+    const int t0 = loA, t1 = hiA;
+    loA = loB; hiA = hiB; loB = t0; hiB = t1;
+  }
+  const int nA = max(0, hiA - loA + 1);
+  const int startB = max(loB, hiA + 1), nB = max(0, hiB - startB + 1);
+  const int nsl = nA + nB;
+  auto slab_at = [&](int u) { return u < nA ? loA + u : startB + (u - nA); };
+  // this warp's first slab
+  unsigned char* my = slabs + warp * AT_STAGE_BYTES;
+  const size_t kvrow0 = (size_t)(b * Hkv + g) * L;
+  int phase = 0;
+  if (lane == 0 && warp < nsl) {
+    const int t = slab_at(warp);
+    tc::mbar_arrive_expect_tx(&bar[warp], AT_STAGE_BYTES);
+    tc::tma_load_3d(my, &kmap, 0, (int)(kvrow0 + (size_t)S * t), 0, &bar[warp]);
+    tc::tma_load_3d(my + 16384, &vmap, 0, (int)(kvrow0 + (size_t)S * t), 0, &bar[warp]);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  // A fragments of the pair's query rows, all 8 k-steps
+  uint32_t qa[8][4];
+  {
+    const int mi = lane >> 3;
+    const uint32_t qrow = smem_u32(qs + (mi & 1) * 2048) + (lane & 7) * 256;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int uq = 2 * ks + (mi >> 1);
+      ldsm_x4(qrow + ((uq ^ (lane & 7)) << 4), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+    }
+  }
+  float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+  float oc[16][4];
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) oc[nt][0] = oc[nt][1] = oc[nt][2] = oc[nt][3] = 0.f;
+  for (int u = warp; u < nsl; u += SW_WARPS) {
+    const int t = slab_at(u);
+    if (!tc::mbar_wait(&bar[warp], (unsigned)phase)) break;
+    phase ^= 1;
+    const uint32_t kst = smem_u32(my), vst = kst + 16384;
+    float sc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    {
+      const int mi = lane >> 3;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t b0, b1, b2, b3;
+          const int key = 16 * np + 8 * (mi >> 1) + (lane & 7), col = 16 * ks + 8 * (mi & 1);
+          ldsm_x4(kst + kv_off(key, col), b0, b1, b2, b3);
+          mma_bf16(sc[2 * np], qa[ks], b0, b1);
+          mma_bf16(sc[2 * np + 1], qa[ks], b2, b3);
+        }
+    }
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hb = e >> 1, p = hb ? pB : pA;
+        const int j = S * t + 8 * nt + 2 * tq + (e & 1);
+        const bool in = (hb == 0 || hasB) && j >= p - w && j <= p + w;
+        const float v = in ? sc[nt][e] * sl2 : -INFINITY;
+        sc[nt][e] = v;
+        mx[hb] = fmaxf(mx[hb], v);
+      }
+    float alpha[2], mnew[2];
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      mx[hb] = fmaxf(mx[hb], __shfl_xor_sync(0xffffffffu, mx[hb], 1));
+      mx[hb] = fmaxf(mx[hb], __shfl_xor_sync(0xffffffffu, mx[hb], 2));
+      mnew[hb] = fmaxf(mrun[hb], mx[hb]);
+      alpha[hb] = mnew[hb] == -INFINITY ? 1.f : fast_exp2(mrun[hb] - mnew[hb]);
+    }
+    float sm[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hb = e >> 1;
+        const float pv = mnew[hb] == -INFINITY ? 0.f : fast_exp2(sc[nt][e] - mnew[hb]);
+        sc[nt][e] = pv;
+        sm[hb] += pv;
+      }
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 1);
+      sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 2);
+      lrun[hb] = lrun[hb] * alpha[hb] + sm[hb];
+      mrun[hb] = mnew[hb];
+    }
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      oc[nt][0] *= alpha[0];
+      oc[nt][1] *= alpha[0];
+      oc[nt][2] *= alpha[1];
+      oc[nt][3] *= alpha[1];
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a[4];
+      a[0] = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
+      a[1] = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
+      a[2] = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+      a[3] = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      const int mi = lane >> 3;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        uint32_t b0, b1, b2, b3;
+        const int key = 16 * kk + 8 * (mi & 1) + (lane & 7), col = 16 * m + 8 * (mi >> 1);
+        ldsm_x4_t(vst + kv_off(key, col), b0, b1, b2, b3);
+        mma_bf16(oc[2 * m], a, b0, b1);
+        mma_bf16(oc[2 * m + 1], a, b2, b3);
+      }
+    }
+    __syncwarp();
+    // next slab of this warp into the same slot
+    const int un = u + SW_WARPS;
+    if (lane == 0 && un < nsl) {
+      const int tn = slab_at(un);
+      tc::fence_proxy_async();
+      tc::mbar_arrive_expect_tx(&bar[warp], AT_STAGE_BYTES);
+      tc::tma_load_3d(my, &kmap, 0, (int)(kvrow0 + (size_t)S * tn), 0, &bar[warp]);
+      tc::tma_load_3d(my + 16384, &vmap, 0, (int)(kvrow0 + (size_t)S * tn), 0, &bar[warp]);
+    }
+  }
+  // ---- fixed-order merge of the warps' states through shared memory (slabs are idle now)
+  __syncthreads();
+  float* part = reinterpret_cast<float*>(slabs) + warp * (16 * 128 + 64);   // [16 rows][128] + m, l
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) {
+    part[gq * 128 + 8 * nt + 2 * tq] = oc[nt][0];
+    part[gq * 128 + 8 * nt + 2 * tq + 1] = oc[nt][1];
+    part[(gq + 8) * 128 + 8 * nt + 2 * tq] = oc[nt][2];
+    part[(gq + 8) * 128 + 8 * nt + 2 * tq + 1] = oc[nt][3];
+  }
+  if (tq == 0) {
+    part[2048 + gq] = mrun[0];
+    part[2048 + 8 + gq] = mrun[1];
+    part[2048 + 16 + gq] = lrun[0];
+    part[2048 + 24 + gq] = lrun[1];
+  }
+  __syncthreads();
+  // thread: one (row of 16, 4 dims) cell per step; rows 0-7 = row A heads, 8-15 = row B
+  const float* p0 = reinterpret_cast<const float*>(slabs);
+  for (int e = tid; e < 16 * 32; e += SW_WARPS * 32) {
+    const int row = e >> 5, d4 = (e & 31) * 4, hd = row & 7, hb = row >> 3;
+    if (hd >= G || (hb == 1 && !hasB)) continue;
+    float M = -INFINITY;
+    for (int x = 0; x < SW_WARPS; ++x) M = fmaxf(M, p0[x * (2048 + 64) + 2048 + hb * 8 + hd]);
+    float Lsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int x = 0; x < SW_WARPS; ++x) {
+      const float* px = p0 + x * (2048 + 64);
+      const float mxx = px[2048 + hb * 8 + hd];
+      if (mxx == -INFINITY) continue;
+      const float f = fast_exp2(mxx - M);
+      Lsum += f * px[2048 + 16 + hb * 8 + hd];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] += f * px[row * 128 + d4 + c];
+    }
+    const int i = hb ? iB : iA, h = g * G + hd;
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + h) * D + d4;
+    const __nv_bfloat162 o01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    const __nv_bfloat162 o23 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&o01);
+    pk.y = *reinterpret_cast<const uint32_t*>(&o23);
+    *reinterpret_cast<uint2*>(orow) = pk;
+    if (lse && d4 == 0) lse[(size_t)(b * Hq + h) * Lq + i] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
+  }
+  (void)C;
+}
+
+// =====================================================================================
 // dec_comb_kernel: one warp per (b, i, h); lane l owns dims 4l .. 4l+3.  Merges the
 // window slab partials (max, sum, unnormalised vector) and, on route layers, the chunk
 // outputs with weights e^{z_c}: one partition, o = sum(weight * vector) / sum(weight).
