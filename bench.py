@@ -30,6 +30,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "route-layer sparse-attn query-tokens/s at 16K-128K; decode-step ms at 128K"
+# DRAM bytes of one rdl_route_attn call on the 16K prefill (window + chunk kernels), from one
+# ncu capture of the current kernels; set to None when either kernel changes.
+ATTN_PREFILL_TRAFFIC = 934.6e6
 UNIT = "query-tokens/s"
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -470,7 +473,10 @@ def main():
         achieved = fl_attn / (call_ms[2] / 1e3) / 1e12
         roof = {"kernel": "rdl_route_attn (window + chunk launches)", "bound": "tensor",
                 "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "frac": achieved / pk["bf16_tflops"], "traffic": ATTN_PREFILL_TRAFFIC,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                  "window_mma_kernel<1> + chunk_tc_kernel, one launch each "
+                                  "(profiles/attn_traffic_route_prefill_16k.md)",
                 "algorithmic_flops": fl_attn, "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
     elif dominant == "rdl_route_score_topk":
         achieved = fl_score / (call_ms[1] / 1e3) / 1e12
