@@ -340,6 +340,48 @@ def stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind):
     torch.cuda.synchronize()
     ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
     assert rdl.rdl_last_device_status() == rdl.OK
+    del g
+
+    def time_graph(fn, reps):
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cs):
+            fn(cs)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(gg, stream=cs):
+                fn(cs)
+        torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            gg.replay()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in evs:
+            flush.zero_()
+            e[0].record(stream)
+            gg.replay()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        return float(np.median([e[0].elapsed_time(e[1]) for e in evs]))
+
+    # the same stack with the window radius of the pages' Table 3 layout (1280) on the 21
+    # sliding-window layers
+    for route, inp, out in layers:
+        if not route:
+            inp.dims.w = 1280
+    ms_w1280 = time_graph(run, args.steps)
+    for route, inp, out in layers:
+        if not route:
+            inp.dims.w = w
+    # dense bidirectional attention of the same 32-query block over the whole 128K cache (one
+    # layer), against the routed layer (score + two-level attention)
+    route0 = next(x for x in layers if x[0])
+    dense_in = api.DeviceInputs(rdl.Dims(B=1, L=L, Lq=Lq, Hq=Hq, Hkv=Hkv, d=d, D=D, r=r, K=K, w=L,
+                                         lam=0.1), "bf16", route0[1].q, route0[1].k, route0[1].v,
+                                route0[1].x, route0[1].w_down, route0[1].w_up, q_pos, None)
+    dense_out = api.alloc_outputs(dense_in.dims, "bf16", dev)
+    ms_dense = time_graph(lambda st: api.swa_attn(dense_in, dense_out, stream=st), args.steps)
+    ms_route = time_graph(lambda st: (api.score_topk(route0[1], route0[2], stream=st),
+                                      api.route_attn(route0[1], route0[2], stream=st)), args.steps)
+    assert rdl.rdl_last_device_status() == rdl.OK
     # bytes the step must move: per route layer as decode_bytes, per window layer its K/V
     # window plus queries and outputs
     by = 0
@@ -349,10 +391,15 @@ def stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind):
         else:
             by += min(L, 64 + 2 * w) * Hkv * 2 * d * 2 + 2 * Lq * 2 * Hq * d
     ach = by / (ms / 1e3) / 1e9
-    del g
     return {"workload": "stack_128k (28 layers: 7 route, 21 sliding window)", "ms_per_step": ms,
             "timing": "one CUDA graph of all 28 layers, median of replays, L2 flushed between",
             "kernels_per_step": launches,
+            "ms_per_step_window_1280": ms_w1280,
+            "dense_vs_route_one_layer": {"dense_bidirectional_ms": ms_dense, "route_ms": ms_route,
+                                         "ratio": ms_dense / ms_route,
+                                         "note": "attention of one layer for the 32-query block "
+                                                 "over the 128K cache; the pages' 172x is the "
+                                                 "whole-model per-token time"},
             "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / pk["hbm_gbs"], "algorithmic_bytes": by,
                          "peak_source": f"hbm_gbs ({pk_kind})"}}
