@@ -644,6 +644,7 @@ constexpr int AT_THREADS = (AT_CONS + 1) * 32;
 constexpr int AT_STAGE_BYTES = 32768;
 constexpr int AT_MAXC = 2048;            // chunks per sequence on this path
 constexpr int AT_QROWS = 32;             // query rows per sequence on this path
+constexpr int AT_SLAB_WORK = 1;          // partition weight of one slab load, in row pairs
 
 // window slabs a row at position p touches: [wlo(p), whi(p)] (w >= 0)
 __device__ __forceinline__ int win_lo(int p, int w) { return max(0, p - w) / S; }
@@ -798,7 +799,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   }
   __syncthreads();
-  // work of slab c: its row pairs plus one slab load; exclusive prefix in chunk order.
+  // work of slab c: its row pairs plus one slab load (weighted AT_SLAB_WORK pairs; heavier
+  // weights measured slower: the pairs of a slab every row selected dominate);
+  // exclusive prefix in chunk order.
   // Slab c belongs to CTA floor(prefix(c) * R / total): contiguous slab ranges of equal work.
   int* scan_ws = misc + 32;                                  // 9 ints
   const int seg = (C + AT_THREADS - 1) / AT_THREADS;
@@ -807,20 +810,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     int local = 0;
     for (int c = s0; c < s1; ++c) {
       const int n = hist[c];
-      local += n > 0 ? (n + 1) / 2 + 1 : 0;
+      local += n > 0 ? (n + 1) / 2 + AT_SLAB_WORK : 0;
     }
     int total;
     int run = cta_excl_scan(local, scan_ws, total);
-    const long long W = total;
+    // run * R < 2^31: at most C slabs x (Lq/2 + K + AT_SLAB_WORK) units x 148 CTAs
     for (int c = s0; c < s1; ++c) {
       const int n = hist[c];
       if (n > 0) {
-        const int owner = (int)(((long long)run * R) / W);
+        const int owner = (run * R) / total;
         if (owner == j) {
           atomicMin(&misc[0], c);
           atomicMax(&misc[1], c);
         }
-        run += (n + 1) / 2 + 1;
+        run += (n + 1) / 2 + AT_SLAB_WORK;
       }
     }
   }
