@@ -117,9 +117,10 @@ int dec_attn_ranges(const rdl_dims* dm) {
   const int r = kSMs / (dm->B * dm->Hkv);
   return r < 1 ? 1 : r;
 }
-// score grid: (ranges, Hq, B) with the range split into TMA boxes through a 3-stage ring
+// score grid: (ranges, Hq, B); each range streams boxes of SC_BOXR summary rows through a
+// ring as deep as shared memory allows (loaded before the dependency wait)
 struct DecScoreGrid {
-  int MT, ranges, ncr, boxr, nbox, nstg, smem;
+  int MT, ranges, ncr, nstg, smem;
 };
 DecScoreGrid dec_score_grid(const rdl_dims* dm) {
   DecScoreGrid gr{};
@@ -131,26 +132,14 @@ DecScoreGrid dec_score_grid(const rdl_dims* dm) {
   ncr = (ncr + 7) & ~7;
   gr.ranges = (C + ncr - 1) / ncr;
   gr.ncr = ncr;
-  // ring depth and box height: as many of the range's summary rows as fit in shared memory
-  // are loaded before the dependency wait
-  const int limit = 232448;
-  int best = -1;
-  for (int nstg = 4; nstg >= 2; --nstg) {
-    const int aux = dec::score_smem(gr.MT, dm->r, 0, nstg, ncr).total;
-    int boxr = ((limit - aux) / (nstg * 512)) & ~7;
-    if (boxr > 256) boxr = 256;
-    const int want = ((ncr + nstg - 1) / nstg + 7) & ~7;
-    if (boxr > want) boxr = want;
-    if (boxr < 8) continue;
-    const int pre = nstg * boxr < ncr ? nstg * boxr : ncr;
-    if (pre > best) {
-      best = pre;
-      gr.nstg = nstg;
-      gr.boxr = boxr;
+  const int nbox = (ncr + dec::SC_BOXR - 1) / dec::SC_BOXR;
+  gr.nstg = 0;
+  for (int nstg = 4; nstg >= 1; --nstg)
+    if (dec::score_smem(gr.MT, dm->r, nstg, ncr).total <= 232448) {
+      gr.nstg = nstg < nbox ? nstg : nbox;
+      break;
     }
-  }
-  gr.nbox = (ncr + gr.boxr - 1) / gr.boxr;
-  gr.smem = dec::score_smem(gr.MT, dm->r, gr.boxr, gr.nstg, ncr).total;
+  gr.smem = gr.nstg > 0 ? dec::score_smem(gr.MT, dm->r, gr.nstg, ncr).total : 0;
   return gr;
 }
 bool use_pdl() {
@@ -298,8 +287,9 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
   const bool split = (dm->flags & RDL_FLAG_SPLIT_SUMMARY) != 0;
   CUtensorMap smap;
   const unsigned long long srows = (unsigned long long)dm->B * dm->Hq * C;
-  if (split ? !make_tmap_split_rows(&smap, summary, srows, (unsigned)gr.boxr)
-            : !make_tmap_f32_rows(&smap, summary, srows, (unsigned)gr.boxr))
+  if (gr.nstg < 1) return RDL_ERR_UNSUPPORTED;
+  if (split ? !make_tmap_split_rows(&smap, summary, srows, (unsigned)dec::SC_BOXR)
+            : !make_tmap_f32_rows(&smap, summary, srows, (unsigned)dec::SC_BOXR))
     return RDL_ERR_CUDA;
   if (res) {
     const int slice = ((dm->D + dec::TK_CL * 64 - 1) / (dec::TK_CL * 64)) * 64;
@@ -327,7 +317,7 @@ rdl_status score_decode(const void* q, const int32_t* q_pos, const void* x, cons
   if (launch_ex(res, kern, dim3(gr.ranges, dm->Hq, dm->B), dim3(dec::SC_WARPS * 32), gr.smem, st, smap, summary,
                  static_cast<const __nv_bfloat16*>(q), q_pos, (const float*)(res ? t : nullptr),
                  static_cast<const __nv_bfloat16*>(w_up), entropy, dm->Lq, dm->L, dm->Hq, res ? dm->r : 0, dm->w, tau,
-                 dm->lambda, gr.ncr, gr.boxr, gr.nbox, gr.nstg, z_all) != cudaSuccess)
+                 dm->lambda, gr.ncr, gr.nstg, z_all) != cudaSuccess)
     return RDL_ERR_CUDA;
   const int G = dm->Hq / dm->Hkv;
   const bool zs = C % 4 == 0 && G * C <= dec::DK_MAXZ;

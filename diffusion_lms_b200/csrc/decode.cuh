@@ -179,37 +179,54 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
 
 // =====================================================================================
 // dec_score_kernel: CTA = (chunk range, query head h, batch b); 16 warps.
-// MT = m-tiles of 16 query rows (rows = Lq <= 16*MT).
+// MT = m-tiles of 16 query rows (NR = 16*MT >= Lq rows).
+// The score tile of one box is D[chunk][row] = s_c . q_res on the 5th-generation tensor
+// cores: M = 128 summary rows straight from the TMA ring (K-major, 128-byte swizzle), K = d,
+// three bf16 split terms: s_hi x [q_hi; q_lo] (N = 2 NR, one operand read for two terms) and
+// s_lo x q_hi (N = NR), in tensor memory (two accumulator sets, so the epilogue of box n
+// overlaps the MMAs of box n + 1).
 // Shared memory:
-//   ring   nstg stages of boxr summary rows, each [4 slices][boxr][32 fp32] with the
-//          128-byte swizzle of the TMA box (16-byte unit ^ row % 8); rewritten in place to
-//          bf16 hi/lo terms once landed
+//   ring   nstg stages of SC_BOXR summary rows; split layout: [4 segments][SC_BOXR][128 B]
+//          (hi 0-63, hi 64-127, lo 0-63, lo 64-127); fp32 layout: [4 slices][SC_BOXR][32 fp32],
+//          rewritten in place to [32 bf16 hi | 32 bf16 lo] per slice row once landed
+//   qsp    q_res split into bf16 hi/lo, K-major with the 128-byte swizzle:
+//          [2 K segments (columns 0-63, 64-127)][q_hi rows 0..NR-1, q_lo rows][128 B]
 //   wup    W_up columns of head h: [r][128] bf16, unit-swizzled (ldmatrix.trans)
-//   qh     q rows of head h: [16*MT][136] bf16 (padded rows)
-//   qsp    q_res rows split into bf16 hi/lo: [16*MT][hi 128 | lo 128], unit-swizzled
-//   ts     t rows: [16*MT][r + 8] fp32
+//   ts     t rows: [NR][r + 8] fp32
+//   hs     entropies of the range; wl/wh: per-row window chunk range (not eligible)
+// Warp roles after the residual: warps 0 and 2 issue the MMAs of the two accumulators
+// (warp-collective), warp 1 refills the ring (one thread), the epilogue warps read the
+// accumulators (TMEM lane quarter = warp % 4) and store the scores: warps 4-11 (two row
+// halves) for split summaries, warps 4-7 for fp32 ones, whose boxes warps 8-15 convert.
 // =====================================================================================
 constexpr int SC_WARPS = 16;
+constexpr int SC_BOXR = 128;                 // summary rows per box = MMA M
+constexpr int SC_BOX_BYTES = SC_BOXR * 512;
+__host__ __device__ constexpr int sc_epi_warps(bool split) { return split ? 8 : 4; }
 struct ScoreSmem {
-  int ring, wup, qh, qsp, ts, hs, ps, bar, total;
+  int ring, qsp, wup, ts, hs, win, bar, total;
 };
-__host__ __device__ inline ScoreSmem score_smem(int MT, int r, int boxr, int nstg, int ncr) {
+__host__ __device__ inline ScoreSmem score_smem(int MT, int r, int nstg, int ncr) {
   ScoreSmem s{};
+  const int NR = 16 * MT;
   int off = 0;
-  s.ring = off; off += nstg * boxr * 512;
+  s.ring = off; off += nstg * SC_BOX_BYTES;
+  s.qsp = off;  off += 4 * NR * 128;
   s.wup = off;  off += (r > 0 ? r : 1) * 256;
-  s.qh = off;   off += MT * 16 * 272;
-  s.qsp = off;  off += MT * 16 * 512;
-  s.ts = off;   off += MT * 16 * (r + 8) * 4;
-  s.hs = off;   off += ((ncr + 3) / 4) * 16;
-  s.ps = off;   off += 64 * 4;
-  s.bar = off;  off += 8 * nstg;
+  s.ts = off;   off += NR * (r + 8) * 4;
+  s.hs = off;   off += ((ncr + 3) & ~3) * 4;
+  s.win = off;  off += 2 * NR * 4;
+  s.bar = off;  off += 8 * (3 * nstg + 5) + 16;
   s.total = off + 1024;       // slack for aligning the base to 1024 bytes
   return s;
 }
 
-// byte offset of 16-byte unit u (0..31: hi 0-15, lo 16-31) of row `row` in a qsp tile
-__device__ __forceinline__ uint32_t qsp_off(int row, int u) { return (uint32_t)(row * 512 + ((u ^ (row & 7)) << 4)); }
+// byte offset of column col (0..255: hi 0-127, lo 128-255) of row `row` in the qsp tile
+// (NR a multiple of 8, so the swizzle row r2 % 8 equals row % 8)
+__device__ __forceinline__ uint32_t qsp_off(int NR, int row, int col) {
+  const int ksg = (col & 127) >> 6, r2 = (col >> 7) * NR + row, within = col & 63;
+  return (uint32_t)(ksg * 2 * NR * 128 + r2 * 128 + (((within >> 3) ^ (r2 & 7)) << 4) + (within & 7) * 2);
+}
 
 template <int MT, bool SPLIT>
 __global__ void __launch_bounds__(SC_WARPS * 32, 1)
@@ -217,21 +234,32 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
                      const float* __restrict__ t, const __nv_bfloat16* __restrict__ w_up,
                      const float* __restrict__ entropy, int Lq, int L, int Hq, int r, int w, float tau,
-                     float lambda, int ncr, int boxr, int nbox, int nstg, float* __restrict__ z_all) {
+                     float lambda, int ncr, int nstg, float* __restrict__ z_all) {
   constexpr int D = 128;
   constexpr int NT = SC_WARPS * 32;
-  constexpr int NG = SC_WARPS / MT;           // warps per m-tile (n-groups)
+  constexpr int NR = 16 * MT;
+  constexpr int NG = SC_WARPS / MT;           // warps per m-tile in the residual (n-groups)
+  constexpr int NPW = 16 / NG;                // residual n-tiles (of 8 columns) per warp
+  // two accumulator sets of 3 NR columns: [s_hi.q_hi | s_hi.q_lo] (2 NR) and s_lo.q_hi (NR)
+  constexpr uint32_t TCOLS = 6 * NR <= 128 ? 128 : (6 * NR <= 256 ? 256 : 512);
   extern __shared__ unsigned char sc_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sc_raw) + 1023) & ~uintptr_t(1023));
-  const ScoreSmem L_ = score_smem(MT, r, boxr, nstg, ncr);
+  const ScoreSmem L_ = score_smem(MT, r, nstg, ncr);
   unsigned char* ring = base + L_.ring;
-  unsigned char* wup = base + L_.wup;
-  unsigned char* qh = base + L_.qh;
   unsigned char* qsp = base + L_.qsp;
+  unsigned char* wup = base + L_.wup;
   float* ts = reinterpret_cast<float*>(base + L_.ts);
   float* hs = reinterpret_cast<float*>(base + L_.hs);
-  int* ps = reinterpret_cast<int*>(base + L_.ps);
+  int* wl = reinterpret_cast<int*>(base + L_.win);
+  int* wh = wl + NR;
   uint64_t* full = reinterpret_cast<uint64_t*>(base + L_.bar);
+  uint64_t* empty = full + nstg;
+  uint64_t* conv = empty + nstg;
+  uint64_t* tfull = conv + nstg;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mdone = tempty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mdone + 1);
+  int* abort_f = reinterpret_cast<int*>(tslot + 1);
   RDL_TRACE_POINT(1, 0);
 
   const int C = L / S;
@@ -244,36 +272,76 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
     grid_dep_wait();
     return;
   }
-  const int nb = min(nbox, (c1 - c0 + boxr - 1) / boxr);
+  const int nb = (c1 - c0 + SC_BOXR - 1) / SC_BOXR;
   const size_t srow0 = (size_t)(b * Hq + h) * C + c0;
   // ---- prologue: only TMA and cp.async.cg loads of inputs (no kernel of this call writes
   // them, and this kernel is launched early only behind dec_t_kernel, which has waited)
+  constexpr int EW = sc_epi_warps(SPLIT);
+  const int npro = min(nb, nstg);     // boxes loaded before the dependency wait
   if (tid == 0) {
-    for (int st = 0; st < nstg; ++st) tc::mbar_init(&full[st], 1);
+    for (int st = 0; st < nstg; ++st) {
+      tc::mbar_init(&full[st], 1);
+      tc::mbar_init(&empty[st], 2);
+      tc::mbar_init(&conv[st], 8);
+    }
+    for (int j = 0; j < 2; ++j) {
+      tc::mbar_init(&tfull[j], 2);
+      tc::mbar_init(&tempty[j], EW);
+    }
+    tc::mbar_init(mdone, 2);
+    *abort_f = 0;
     tc::mbar_fence_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    for (int bx = 0; bx < nb && bx < nstg; ++bx) {
-      tc::mbar_arrive_expect_tx(&full[bx], (unsigned)boxr * 512u);
-      tc::tma_load_3d(ring + bx * boxr * 512, &smap, 0, (int)(srow0 + (size_t)bx * boxr), 0, &full[bx]);
+    for (int bx = 0; bx < npro; ++bx) {
+      tc::mbar_arrive_expect_tx(&full[bx], (unsigned)SC_BOX_BYTES);
+      tc::tma_load_3d(ring + bx * SC_BOX_BYTES, &smap, 0, (int)(srow0 + (size_t)bx * SC_BOXR), 0, &full[bx]);
     }
   }
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_alloc(tslot, TCOLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tslot;
+  int n_issued = npro;                // boxes issued (prologue, then refills by thread 32)
   for (int e = tid; e < r * 16; e += NT) {
     const int kk = e >> 4, u = e & 15;
     cp_async16(smem_u32(wup + kk * 256 + ((u ^ (kk & 7)) << 4)), w_up + (size_t)kk * Hq * D + h * D + u * 8);
   }
-  for (int e = tid; e < Lq * 16; e += NT) {
-    const int i = e >> 4, u = e & 15;
-    cp_async16(smem_u32(qh + i * 272 + u * 16), q + ((size_t)(b * Lq + i) * Hq + h) * D + u * 8);
-  }
   cp_async_commit();
+  // the q values this thread adds to its residual fragment (rows row0/row1, NPW n-tiles)
+  __nv_bfloat162 qv[NPW][2];
+  {
+    const int row0 = mw * 16 + gq;
+#pragma unroll
+    for (int n = 0; n < NPW; ++n) {
+      const int col = (ng * NPW + n) * 8 + 2 * tq;
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = row0 + 8 * hr;
+        qv[n][hr] = row < Lq ? *reinterpret_cast<const __nv_bfloat162*>(q + ((size_t)(b * Lq + row) * Hq + h) * D + col)
+                             : __floats2bfloat162_rn(0.f, 0.f);
+      }
+    }
+  }
   for (int j = tid; j < c1 - c0; j += NT) hs[j] = __ldcg(entropy + (size_t)(b * Hq + h) * C + c0 + j);
-  if (tid < MT * 16) ps[tid] = tid < Lq ? (q_pos ? __ldcg(q_pos + (size_t)b * Lq + tid) : tid) : INT_MIN;
+  if (tid < NR) {
+    // window chunk range of row tid: chunks wl..wh are not eligible (empty when wl > wh)
+    const int p = tid < Lq ? (q_pos ? __ldcg(q_pos + (size_t)b * Lq + tid) : tid) : INT_MIN;
+    if (w < 0 || p == INT_MIN) {
+      wl[tid] = 1;
+      wh[tid] = 0;
+    } else {
+      wl[tid] = p - w <= 0 ? INT_MIN : (p - w) / S;
+      wh[tid] = (p + w) / S;
+    }
+  }
   // rows beyond the ring: pulled into L2 now, loaded into the ring when a stage frees
   for (int bx = nstg + warp; bx < nb; bx += SC_WARPS) {
-    const char* src = reinterpret_cast<const char*>(smap_base) + (srow0 + (size_t)bx * boxr) * 512;
-    const int bytes = min(boxr, (c1 - c0) - bx * boxr) * 512;
+    const char* src = reinterpret_cast<const char*>(smap_base) + (srow0 + (size_t)bx * SC_BOXR) * 512;
+    const int bytes = min(SC_BOXR, (c1 - c0) - bx * SC_BOXR) * 512;
     for (int off = lane * 4096; off < bytes; off += 32 * 4096)
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src + off), "r"(min(4096, bytes - off))
                    : "memory");
@@ -292,9 +360,8 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
   cp_async_commit();
 
   // ---- q_res = q + t W_up for this warp's m-tile and n-group (tensor cores, t split),
-  // written straight into the split hi/lo tile
+  // written straight into the split hi/lo operand tile
   {
-    constexpr int NPW = 16 / NG;              // n-tiles (of 8 columns) per warp
     float ua[NPW][4];
 #pragma unroll
     for (int n = 0; n < NPW; ++n) ua[n][0] = ua[n][1] = ua[n][2] = ua[n][3] = 0.f;
@@ -334,129 +401,189 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int row = mw * 16 + gq + 8 * hr;
-        const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qh + row * 272 + col * 2));
+        const float2 qf = __bfloat1622float2(qv[n][hr]);
         uint32_t hi, lo;
         split2(qf.x + ua[n][2 * hr], qf.y + ua[n][2 * hr + 1], hi, lo);
-        // unit col/8 holds columns col/8*8 .. +7; this pair is word (col % 8) / 2 of it
-        *reinterpret_cast<uint32_t*>(qsp + qsp_off(row, col >> 3) + (col & 7) * 2) = hi;
-        *reinterpret_cast<uint32_t*>(qsp + qsp_off(row, 16 + (col >> 3)) + (col & 7) * 2) = lo;
+        *reinterpret_cast<uint32_t*>(qsp + qsp_off(NR, row, col)) = hi;
+        *reinterpret_cast<uint32_t*>(qsp + qsp_off(NR, row, 128 + col)) = lo;
       }
     }
   }
+  tc::fence_proxy_async();            // the operand tile is read by the tensor cores
   __syncthreads();
   RDL_TRACE_POINT(1, 3);
-  int wlo[2], whi[2];   // window chunk range of the warp's two rows: chunks wlo..whi are not eligible
-  const int irow[2] = {mw * 16 + gq, mw * 16 + gq + 8};
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    const int p = ps[irow[hr]];
-    if (w < 0 || p == INT_MIN) {
-      wlo[hr] = 1;
-      whi[hr] = 0;
-    } else {
-      wlo[hr] = p - w <= 0 ? INT_MIN : (p - w) / S;     // chunk containing p - w (or none below 0)
-      whi[hr] = (p + w) / S;
-    }
-  }
-  // ---- scores over the range, box by box as the TMA loads land.  An fp32 box is first
-  // rewritten in place (a box of split-layout summaries is used as it lands): every 128-byte segment (32 fp32 of one summary row) becomes 32 bf16
-  // hi terms (logical 16-byte units 0-3) and 32 bf16 lo terms (units 4-7), x = hi + lo to
-  // ~2^-17, keeping the unit ^ (row % 8) swizzle so the fragment loads stay conflict-free.
-  const int ntb = boxr / 8;
-  for (int bx = 0; bx < nb; ++bx) {
-    const int st = bx % nstg;
-    if (!tc::mbar_wait(&full[st], (unsigned)(bx / nstg) & 1u)) break;
-    if (bx == 0) RDL_TRACE_POINT(1, 4);
-    if (bx == 1) RDL_TRACE_POINT(1, 6);
-    if (bx == nb - 1) RDL_TRACE_POINT(1, 7);
-    unsigned char* stg = ring + st * boxr * 512;
-    for (int seg = tid; !SPLIT && seg < 4 * boxr; seg += NT) {
-      const int rr = seg % boxr;
-      unsigned char* sp = stg + (seg / boxr) * boxr * 128 + rr * 128;
-      const int sw = rr & 7;
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const float4*>(sp + ((u ^ sw) << 4));
-      uint32_t hi[16], lo[16];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        split2(v[u].x, v[u].y, hi[2 * u], lo[2 * u]);
-        split2(v[u].z, v[u].w, hi[2 * u + 1], lo[2 * u + 1]);
+
+  if (warp == 0 || warp == 2) {
+    // ---------------- MMA issuers (warp-collective, one elected lane issues): warp 0 the
+    // s_hi x [q_hi; q_lo] accumulator, warp 2 the s_lo x q_hi one
+    const bool hi_set = warp == 0;
+    const uint32_t idesc = hi_set ? tc::idesc_bf16(128, 2 * NR, false, false) : tc::idesc_bf16(128, NR, false, false);
+    const uint64_t dq0 = tc::sdesc(smem_u32(qsp), 16, 1024);
+    const uint64_t qks = (uint64_t)((2 * NR * 128) >> 4);        // K segment of the q tile
+    const uint64_t aseg = (uint64_t)((SC_BOXR * 128) >> 4);      // segment of a box
+    bool issued = false;
+    for (int bx = 0; bx < nb; ++bx) {
+      const int st = bx % nstg, buf = bx & 1;
+      const unsigned ph = (unsigned)(bx / nstg) & 1u;
+      const bool ok = tc::mbar_wait(SPLIT ? &full[st] : &conv[st], ph) &&
+                      tc::mbar_wait(&tempty[buf], ((unsigned)(bx >> 1) & 1u) ^ 1u) && !*(volatile int*)abort_f;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) *(volatile int*)abort_f = 1;
+        break;
       }
+      if (bx == 0) RDL_TRACE_POINT(1, 4);
+      if (bx == 1) RDL_TRACE_POINT(1, 6);
+      if (bx == nb - 1) RDL_TRACE_POINT(1, 7);
+      tc::tc_fence_after();
+      const uint64_t da0 = tc::sdesc(smem_u32(ring + st * SC_BOX_BYTES), 16, 1024);
+      const uint32_t dt = tbase + (uint32_t)(buf * 3 * NR + (hi_set ? 0 : 2 * NR));
+      if (SPLIT) {
+        // box segments: 0, 1 = s hi (columns 0-63, 64-127), 2, 3 = s lo
+        const int sa = hi_set ? 0 : 2;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        *reinterpret_cast<uint4*>(sp + ((u ^ sw) << 4)) = make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
-        *reinterpret_cast<uint4*>(sp + (((4 + u) ^ sw) << 4)) =
-            make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16_ss_warp(dt, da0 + (sa + j) * aseg + 2 * k, dq0 + j * qks + 2 * k, idesc, (j | k) != 0);
+      } else {
+        // slice s holds columns 32s..32s+31 as [16 hi | 16 hi | 16 lo | 16 lo] (32 B each)
+        const int ao = hi_set ? 0 : 4;
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const uint64_t bq = dq0 + (uint64_t)(sl >> 1) * qks + (uint64_t)((sl & 1) * 4 + 2 * k);
+            tc::mma_bf16_ss_warp(dt, da0 + sl * aseg + ao + 2 * k, bq, idesc, (sl | k) != 0);
+          }
       }
+      tc::mma_commit_warp(&tfull[buf]);
+      tc::mma_commit_warp(&empty[st]);
+      issued = true;
     }
-    __syncthreads();
-    const uint32_t stu = smem_u32(stg);
-    const int cb = c0 + bx * boxr;
-    // this warp's n-tiles of the box: ng, ng + NG, ... (at most 2 for NG >= ntb / 2)
-    for (int nt0 = ng; nt0 < ntb; nt0 += 2 * NG) {
-      const int nt1 = nt0 + NG;
-      const bool two = nt1 < ntb;
-      float a0[2][4], a1[2][4], a2[2][4];
+    // every MMA issued has completed before the tensor memory is released
+    if (issued) tc::mma_commit_warp(mdone); else tc::mbar_arrive_warp(mdone);
+    (void)tc::mbar_wait(mdone, 0);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- ring refills (the stage's MMAs have completed)
+    if (lane == 0) {
+      for (int bx = nstg; bx < nb; ++bx) {
+        const int st = bx % nstg;
+        if (!tc::mbar_wait(&empty[st], (unsigned)(bx / nstg - 1) & 1u) || *(volatile int*)abort_f) {
+          *(volatile int*)abort_f = 1;
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&full[st], (unsigned)SC_BOX_BYTES);
+        tc::tma_load_3d(ring + st * SC_BOX_BYTES, &smap, 0, (int)(srow0 + (size_t)bx * SC_BOXR), 0, &full[st]);
+        ++n_issued;
+      }
+      // the last box issued into each stage has landed before the CTA may exit
+      for (int bx = max(0, n_issued - nstg); bx < n_issued; ++bx)
+        (void)tc::mbar_wait(&full[bx % nstg], (unsigned)(bx / nstg) & 1u);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 4 + EW) {
+    // ---------------- epilogue: lanes 32 (warp % 4) .. + 31 of the accumulator = chunks;
+    // rows [r0, r0 + RPW) of them
+    constexpr int RPW = NR * 4 / EW;
+    constexpr int CH = RPW < 16 ? RPW : 16;
+    const int quad = warp & 3, r0 = ((warp - 4) >> 2) * RPW;
+    // chunks outside [wmin, wmax] are eligible for every row (the usual case: the rows of a
+    // block share one narrow window), so the per-row test runs only inside it
+    int wmin = INT_MAX, wmax = INT_MIN;
+    for (int i = 0; i < Lq; ++i)
+      if (wl[i] <= wh[i]) {
+        wmin = min(wmin, wl[i]);
+        wmax = max(wmax, wh[i]);
+      }
+    for (int bx = 0; bx < nb; ++bx) {
+      const int buf = bx & 1;
+      const bool ok = tc::mbar_wait(&tfull[buf], (unsigned)(bx >> 1) & 1u) && !*(volatile int*)abort_f;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) *(volatile int*)abort_f = 1;
+        break;
+      }
+      const int c = c0 + bx * SC_BOXR + 32 * quad + lane;
+      // eligibility of (row, c) as a bit mask and the entropy term, read before any store
+      unsigned long long em = ~0ull;
+      if (c >= wmin && c <= wmax) {
+        em = 0ull;
+        for (int i = 0; i < NR; ++i)
+          if (c < wl[i] || c > wh[i]) em |= 1ull << i;
+      }
+      const float eh = c < c1 ? lambda * hs[c - c0] : 0.f;
+      float* zc = z_all + (size_t)(b * Hq + h) * Lq * C + c;
+      tc::tc_fence_after();
+      const uint32_t ta = tc::taddr(tbase, 32 * quad, buf * 3 * NR);
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
+      for (int i0 = r0; i0 < r0 + RPW; i0 += CH) {
+        float vh[CH], vl[CH], vs[CH];
+        if constexpr (CH == 16) {
+          tc::tmem_ld16(ta + i0, vh);
+          tc::tmem_ld16(ta + NR + i0, vl);
+          tc::tmem_ld16(ta + 2 * NR + i0, vs);
+        } else {
+          tc::tmem_ld8(ta + i0, vh);
+          tc::tmem_ld8(ta + NR + i0, vl);
+          tc::tmem_ld8(ta + 2 * NR + i0, vs);
+        }
+        tc::tmem_wait_ld();
+        if (i0 + CH >= r0 + RPW) {
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&tempty[buf]);
+        }
+        if (c < c1) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) a0[x][e] = a1[x][e] = a2[x][e] = 0.f;
-      const int mj = lane >> 3;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t ahi[4], alo[4];
-        const int ra = mw * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), ua = 2 * ks + (lane >> 4);
-        ldsm_x4(smem_u32(qsp + qsp_off(ra, ua)), ahi[0], ahi[1], ahi[2], ahi[3]);
-        ldsm_x4(smem_u32(qsp + qsp_off(ra, 16 + ua)), alo[0], alo[1], alo[2], alo[3]);
-        // converted fp32 box: slice ks/2, units hi 0-3 / lo 4-7; split-layout box: segments
-        // hi (ks/4), lo (2 + ks/4), units 2 (ks % 4) + {0, 1}
-        const int un = SPLIT ? 2 * (ks & 3) + (mj & 1) : (mj >= 2 ? 4 : 0) + ((16 * ks) & 31) / 8 + (mj & 1);
-        const int sg = SPLIT ? (mj >= 2 ? 2 : 0) + (ks >> 2) : (ks >> 1);
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (x == 1 && !two) break;
-          const int rl = (x ? nt1 : nt0) * 8 + (lane & 7);
-          uint32_t bh0, bh1, bl0, bl1;
-          ldsm_x4(stu + sg * boxr * 128 + rl * 128 + ((un ^ (rl & 7)) << 4), bh0, bh1, bl0, bl1);
-          mma_bf16(a0[x], ahi, bh0, bh1);
-          mma_bf16(a1[x], ahi, bl0, bl1);
-          mma_bf16(a2[x], alo, bh0, bh1);
+          for (int e = 0; e < CH; ++e) {
+            const int i = i0 + e;
+            if (i >= Lq) break;
+            const float acc = vh[e] + (vl[e] + vs[e]);
+            __stcg(zc + (size_t)i * C, ((em >> i) & 1ull) ? tau * acc - eh : -INFINITY);
+          }
         }
       }
+    }
+  } else if (!SPLIT && warp >= 8) {
+    // ---------------- fp32 boxes: rewrite every 128-byte slice row (32 fp32) in place as
+    // 32 bf16 hi terms then 32 bf16 lo terms (x = hi + lo to ~2^-17), keeping the swizzle
+    const int ct = tid - 256;
+    for (int bx = 0; bx < nb; ++bx) {
+      const int st = bx % nstg;
+      if (!tc::mbar_wait(&full[st], (unsigned)(bx / nstg) & 1u) || *(volatile int*)abort_f) {
+        *(volatile int*)abort_f = 1;
+        break;
+      }
+      unsigned char* stg = ring + st * SC_BOX_BYTES;
+      for (int seg = ct; seg < 4 * SC_BOXR; seg += 256) {
+        const int rr = seg % SC_BOXR;
+        unsigned char* sp = stg + (seg / SC_BOXR) * SC_BOXR * 128 + rr * 128;
+        const int sw = rr & 7;
+        float4 vv[8];
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (x == 1 && !two) break;
-        const int cc = cb + (x ? nt1 : nt0) * 8 + 2 * tq;
+        for (int u = 0; u < 8; ++u) vv[u] = *reinterpret_cast<const float4*>(sp + ((u ^ sw) << 4));
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int i = irow[hr];
-          if (i >= Lq) continue;
-          float z[2];
+        for (int u = 0; u < 8; ++u) {
+          split2(vv[u].x, vv[u].y, hi[2 * u], lo[2 * u]);
+          split2(vv[u].z, vv[u].w, hi[2 * u + 1], lo[2 * u + 1]);
+        }
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = cc + e;
-            const float acc = a0[x][2 * hr + e] + (a1[x][2 * hr + e] + a2[x][2 * hr + e]);
-            const bool elig = c < c1 && (c < wlo[hr] || c > whi[hr]);
-            z[e] = elig ? tau * acc - lambda * hs[c - c0] : -INFINITY;
-          }
-          float* zr = z_all + ((size_t)(b * Hq + h) * Lq + i) * C;
-          if (cc + 1 < c1 && ((C & 1) == 0)) {
-            *reinterpret_cast<float2*>(zr + cc) = make_float2(z[0], z[1]);
-          } else {
-            if (cc < c1) zr[cc] = z[0];
-            if (cc + 1 < c1) zr[cc + 1] = z[1];
-          }
+        for (int u = 0; u < 4; ++u) {
+          *reinterpret_cast<uint4*>(sp + ((u ^ sw) << 4)) = make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+          *reinterpret_cast<uint4*>(sp + (((4 + u) ^ sw) << 4)) =
+              make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
         }
       }
-    }
-    __syncthreads();                       // stage consumed by every warp
-    if (tid == 0 && bx + nstg < nb) {
       tc::fence_proxy_async();
-      tc::mbar_arrive_expect_tx(&full[st], (unsigned)boxr * 512u);
-      tc::tma_load_3d(ring + st * boxr * 512, &smap, 0, (int)(srow0 + (size_t)(bx + nstg) * boxr), 0, &full[st]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&conv[st]);
     }
   }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 0) tc::tmem_dealloc(tbase, TCOLS);
   RDL_TRACE_POINT(1, 5);
 }
 
