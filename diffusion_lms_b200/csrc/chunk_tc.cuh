@@ -18,8 +18,9 @@
 //   The home accumulators O^T [128 lanes x 45*8 columns] stay in TMEM for the whole tile;
 //   the epilogue adds the window part and writes o once.
 //
-// Costs that shape the design (measured on B200): a tcgen05.mma takes about the same issue
-// time (~50 cycles) for every shape up to N = 64, so a pass is bounded by its 12 MMAs; a
+// Costs that shape the design (measured on B200): a tcgen05.mma issued by a converged warp
+// takes about the same time (~63 cycles) for every shape up to N = 128 (~144 from a
+// single-lane branch), so a pass is bounded by its 12 MMAs; a
 // TMA instruction takes ~130 cycles to issue whatever its box size, so loads are made as
 // large as possible: K and V one 3D box each, and the Q rows of a pass one 4D box per run
 // of consecutive query tokens (the buckets are sorted so that runs are long).  S and T
@@ -28,8 +29,8 @@
 //
 // Warp roles (640 threads):
 //   warp 0        Q producer (TMA, lane 0)
-//   warp 1        TMEM owner, issuer of the S MMAs
-//   warp 2        issuer of the PV MMAs
+//   warp 1        TMEM owner, issuer of the S MMAs (warp-collective issue)
+//   warp 2        issuer of the PV MMAs (warp-collective issue)
 //   warps 3-10    two softmax groups (even / odd passes), one warp per TMEM lane quarter.
 //                 An M=64 result occupies lanes 0-15 of each quarter; the 16x256b load
 //                 shape spreads them over all 32 threads (thread t: rows t/4 and t/4+8,
@@ -370,69 +371,71 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     }
   }
   // ---------------------------------------------------------------- S MMAs
+  // (the whole warp runs the issue loop; one elected lane issues: warp-uniform issue keeps
+  // the descriptors in uniform registers)
   else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
-      const uint32_t dS = tbase + (uint32_t)CT_SCOL;
-      int k = 0;
-      bool ok = true, issued = false;
-      for (int u = 0; u < U && ok; ++u) {
-        const int n = uni[u] >> 24, slot = u % CT_NSLOT;
-        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
-        const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
-        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
-          const int ab = k % CT_NA, sb = k & 1;
-          if (!ct_wait(&B.afull[ab], (k / CT_NA) & 1, abort_flag) ||
-              !ct_wait(B.sempty, (k & 1) ^ 1, abort_flag)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint64_t da = dA0 + (uint64_t)((ab * 16384) >> 4);
+    const uint32_t idesc_s = tc::idesc_bf16(64, 64, false, false);
+    const uint32_t dS = tbase + (uint32_t)CT_SCOL;
+    int k = 0;
+    bool ok = true, issued = false;
+    for (int u = 0; u < U && ok; ++u) {
+      const int n = __shfl_sync(0xffffffffu, (int)(uni[u] >> 24), 0), slot = u % CT_NSLOT;
+      if (!__all_sync(0xffffffffu, ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag))) break;
+      const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
+      for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+        const int ab = k % CT_NA, sb = k & 1;
+        const bool w_ok = ct_wait(&B.afull[ab], (k / CT_NA) & 1, abort_flag) &&
+                          ct_wait(B.sempty, (k & 1) ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint64_t da = dA0 + (uint64_t)((ab * 16384) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {      // K steps of 16: halves at +1 KB (Q) / +8 KB (K)
-            const uint64_t qoff = (uint64_t)((ks >> 2) * 64 + (ks & 3) * 2);
-            const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);
-            tc::mma_bf16_ss(dS, da + qoff, dk + koff, idesc_s, ks > 0);
-          }
-          tc::mma_commit(&B.sfull[sb]);
-          tc::mma_commit(&B.aempty[ab]);
-          if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // K of this chunk done
-          issued = true;
+        for (int ks = 0; ks < 8; ++ks) {      // K steps of 16: halves at +1 KB (Q) / +8 KB (K)
+          const uint64_t qoff = (uint64_t)((ks >> 2) * 64 + (ks & 3) * 2);
+          const uint64_t koff = (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2);
+          tc::mma_bf16_ss_warp(dS, da + qoff, dk + koff, idesc_s, ks > 0);
         }
+        tc::mma_commit_warp(&B.sfull[sb]);
+        tc::mma_commit_warp(&B.aempty[ab]);
+        if (p0 + CT_QP >= n) tc::mma_commit_warp(&B.empty[slot]);     // K of this chunk done
+        issued = true;
       }
-      if (issued) tc::mma_commit(&B.done[0]); else tc::mbar_arrive(&B.done[0]);
-      tc::mbar_wait(&B.done[0], 0);          // bounded; not cut short by an abort
     }
+    if (issued) tc::mma_commit_warp(&B.done[0]); else tc::mbar_arrive_warp(&B.done[0]);
+    tc::mbar_wait(&B.done[0], 0);          // bounded; not cut short by an abort
+    __syncwarp();
   }
   // ---------------------------------------------------------------- PV MMAs
   else if (warp == 2) {
-    if (lane == 0) {
-      const uint32_t dT = tbase + (uint32_t)CT_TCOL;
-      int k = 0;
-      bool ok = true, issued = false;
-      for (int u = 0; u < U && ok; ++u) {
-        const int n = uni[u] >> 24, slot = u % CT_NSLOT;
-        if (!ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag)) break;
-        const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
-        for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
-          const int nq = min(CT_QP, n - p0), pb = k & 1;
-          if (!ct_wait(&B.pfull[pb], (k >> 1) & 1, abort_flag) ||
-              !ct_wait(B.tempty, (k & 1) ^ 1, abort_flag)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint64_t bd0 = dP0 + (uint64_t)((pb * 8192) >> 4);
-          // N rounded up to a multiple of 16; P rows past 8*nq are zero
-          const uint32_t idesc_pv = tc::idesc_bf16(128, 16 * ((nq + 1) >> 1), true, false);
-          tc::mma_bf16_ss(dT, ad0, bd0, idesc_pv, false);
-          tc::mma_bf16_ss(dT, ad0 + 128, bd0 + 2, idesc_pv, true);
-          tc::mma_bf16_ss(dT, ad0 + 256, bd0 + 4, idesc_pv, true);
-          tc::mma_bf16_ss(dT, ad0 + 384, bd0 + 6, idesc_pv, true);
-          tc::mma_commit(B.tfull);
-          tc::mma_commit(&B.pempty[pb]);
-          if (p0 + CT_QP >= n) tc::mma_commit(&B.empty[slot]);     // V of this chunk done
-          issued = true;
-        }
+    const uint32_t dT = tbase + (uint32_t)CT_TCOL;
+    int k = 0;
+    bool ok = true, issued = false;
+    for (int u = 0; u < U && ok; ++u) {
+      const int n = __shfl_sync(0xffffffffu, (int)(uni[u] >> 24), 0), slot = u % CT_NSLOT;
+      if (!__all_sync(0xffffffffu, ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag))) break;
+      const uint64_t ad0 = dV0 + (uint64_t)((slot * 32768) >> 4);
+      for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
+        const int nq = min(CT_QP, n - p0), pb = k & 1;
+        const bool w_ok = ct_wait(&B.pfull[pb], (k >> 1) & 1, abort_flag) &&
+                          ct_wait(B.tempty, (k & 1) ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint64_t bd0 = dP0 + (uint64_t)((pb * 8192) >> 4);
+        // N rounded up to a multiple of 16; P rows past 8*nq are zero
+        const uint32_t idesc_pv = tc::idesc_bf16(128, 16 * ((nq + 1) >> 1), true, false);
+        tc::mma_bf16_ss_warp(dT, ad0, bd0, idesc_pv, false);
+        tc::mma_bf16_ss_warp(dT, ad0 + 128, bd0 + 2, idesc_pv, true);
+        tc::mma_bf16_ss_warp(dT, ad0 + 256, bd0 + 4, idesc_pv, true);
+        tc::mma_bf16_ss_warp(dT, ad0 + 384, bd0 + 6, idesc_pv, true);
+        tc::mma_commit_warp(B.tfull);
+        tc::mma_commit_warp(&B.pempty[pb]);
+        if (p0 + CT_QP >= n) tc::mma_commit_warp(&B.empty[slot]);     // V of this chunk done
+        issued = true;
       }
-      if (issued) tc::mma_commit(&B.done[1]); else tc::mbar_arrive(&B.done[1]);
-      tc::mbar_wait(&B.done[1], 0);
     }
+    if (issued) tc::mma_commit_warp(&B.done[1]); else tc::mbar_arrive_warp(&B.done[1]);
+    tc::mbar_wait(&B.done[1], 0);
+    __syncwarp();
   }
   // ---------------------------------------------------------------- softmax groups
   else if (warp <= 10) {
