@@ -182,7 +182,8 @@ ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   w.zeta = off;
   if (!dec_score_ok(dm, dt)) off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
   if (dec_score_ok(dm, dt)) {
-    w.t = off;     off += align256(sizeof(float) * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
+    // the hidden-slice partials of t, summed by the scorer
+    w.t = off;     off += align256(sizeof(float) * dec::TK_CL * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
   } else if (fast_score(dm, dt)) {
     w.tt = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Lq * 2 * dm->r);
     w.sb = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Hq * C * (2 * dm->d + 2 * dm->r));

@@ -4,21 +4,22 @@
 // organised for this shape, where the bytes that must come from HBM are the cached
 // summaries (fp32, read once) and the K/V slabs of the selected chunks:
 //
-//   dec_t_kernel      t = x W_down, one cluster of 8 CTAs: each CTA contracts one slice of
-//                     the hidden size on tensor cores, the partial products are summed in a
-//                     fixed order through distributed shared memory.
+//   dec_t_kernel      t = x W_down: 8 CTAs, each contracts one slice of the hidden size on
+//                     tensor cores and writes its partial; the scorer sums the partials in
+//                     a fixed order.
 //   dec_score_kernel  CTA = (batch, query head, chunk range).  Before its dependency wait it
-//                     starts TMA loads of its summary rows into shared memory, so the one
-//                     pass over the summaries overlaps the residual.  Then
-//                     q_res = q + t W_up for its head (tensor cores) and the split-bf16
-//                     score z = tau q_res.s - lambda H over the range.
+//                     starts TMA loads of its summary rows into shared memory (and pulls the
+//                     rest into L2), so the one pass over the summaries overlaps the
+//                     residual.  Then q_res = q + t W_up for its head and the split-bf16
+//                     score z = tau q_res.s - lambda H on tcgen05 tensor cores (summary rows
+//                     as the M = 128 operand, accumulators in tensor memory).
 //   dec_topk_kernel   CTA = (batch, query row, KV group): zeta = max over the group's heads,
-//                     exact top-K (radix select), per-head scores of the selected chunks.
-//   dec_attn_kernel   chunk-major: a CTA owns one (batch, group, chunk range), finds in idx
-//                     every (row, slot) that selected a chunk of its range, streams each
-//                     selected chunk's K/V once through a TMA ring and computes the
-//                     second-level softmax output of every row that selected it; window CTAs
-//                     run the bidirectional local window of 4 rows each.
+//                     exact top-K (candidate filter, radix select on heavy ties), per-head
+//                     scores of the selected chunks.
+//   dec_attn_kernel   chunk-major: the CTAs of a (batch, group) split the 64-key slabs that
+//                     some row needs (a selected chunk or a window slab) into contiguous
+//                     ranges of equal work, stream each slab's K/V once through a TMA ring
+//                     and compute every task on it (two rows per warp on tensor cores).
 //   dec_comb_kernel   one partition per (row, head): Z = e^lambda_loc + sum_c e^{z_c} and
 //                     o = (e^lambda_loc o_loc + sum_c e^{z_c} o_c) / Z, in a fixed order.
 //
@@ -27,7 +28,6 @@
 // allows its dependent to launch only after that wait, so the early start of a dependent
 // never reads data older than the call's own inputs.
 #pragma once
-#include <cooperative_groups.h>
 #include "common.cuh"
 #include "tc.cuh"
 #include "score.cuh"
@@ -39,8 +39,6 @@
 
 namespace rdl {
 namespace dec {
-
-namespace cg = cooperative_groups;
 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
@@ -61,22 +59,25 @@ __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
 }
 
 // =====================================================================================
-// dec_t_kernel: t[M, r] = x[M, D] W_down[D, r] (bf16 inputs, exact products, fp32 sums).
-// One cluster of 8 CTAs; CTA `rank` owns hidden slice [rank*slice, rank*slice + slice).
+// dec_t_kernel: partial t of a hidden slice, tp[rank][M, r] = x[M, slice] W_down[slice, r]
+// (bf16 inputs, exact products, fp32 sums).  8 CTAs; CTA `rank` owns hidden slice
+// [rank*slice, rank*slice + slice).  The scorer sums the 8 partials in rank order (the
+// same result on every run); no cross-CTA barrier, which under the scorer's early summary
+// stream measured 2-3 us.
 // =====================================================================================
 constexpr int TK_CL = 8;
 constexpr int TK_KMAX = 512;                                // hidden columns per load batch
 
 // shared memory of dec_t_kernel for `rows` (multiple of 16) query rows, rank r and a batch
 // of kc hidden columns (multiple of 64): per 64-column block, x [rows][128 B] and
-// W_down [64][128 B] per 64 columns of r (TMA boxes, 128-byte swizzle); partial t [rows][r].
+// W_down [64][128 B] per 64 columns of r (TMA boxes, 128-byte swizzle).
 __host__ __device__ inline int tk_smem(int rows, int r, int kc) {
-  return 1024 + (kc / 64) * (rows * 128 + (r / 64) * 8192) + rows * r * 4 + 16;
+  return 1024 + (kc / 64) * (rows * 128 + (r / 64) * 8192) + 16;
 }
 
-__global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
+__global__ void __launch_bounds__(256)
     dec_t_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, int M,
-                 int D, int r, int kc, float* __restrict__ t) {
+                 int D, int r, int kc, float* __restrict__ tp) {
   extern __shared__ unsigned char tk_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(tk_raw) + 1023) & ~uintptr_t(1023));
   RDL_TRACE_POINT(0, 0);
@@ -86,8 +87,7 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
   const int xblk = rows * 128, wblk = nnb * 8192;
   unsigned char* xs = base;                                    // [nkb][rows][128 B]
   unsigned char* ws = xs + nkb * xblk;                         // [nkb][nnb][64][128 B]
-  float* part = reinterpret_cast<float*>(ws + nkb * wblk);     // [rows][r]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(part + rows * r);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(ws + nkb * wblk);
   if (tid == 0) {
     tc::mbar_init(bar, 1);
     tc::mbar_fence_init();
@@ -96,8 +96,7 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
   grid_dep_wait();
   grid_dep_launch();
   RDL_TRACE_POINT(0, 1);
-  cg::cluster_group cl = cg::this_cluster();
-  const int rank = (int)cl.block_rank();
+  const int rank = blockIdx.x;
   const int slice = ((D + TK_CL * 64 - 1) / (TK_CL * 64)) * 64;
   const int k0 = min(D, rank * slice), k1 = min(D, k0 + slice);
   const int npairs = r / 16, ntask = Mt * npairs;
@@ -142,12 +141,9 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
     __syncthreads();
   }
   RDL_TRACE_POINT(0, 3);
-  // push reduction: CTA `rank` stores its partial of row block j straight into CTA j's
-  // shared memory (recv[rank]); one cluster barrier, then every CTA sums its own block in
-  // rank order, so the result is the same on every run
+  // this CTA's partial straight from the accumulators
   const int gq = lane >> 2, tq = lane & 3;
-  const int rows_per = (M + TK_CL - 1) / TK_CL;
-  float* recv = part;                                          // [TK_CL][rows_per][r]
+  float* tr = tp + (size_t)rank * M * r;
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int task = warp + 8 * a;
@@ -157,22 +153,12 @@ __global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(256)
     for (int hr = 0; hr < 2; ++hr) {
       const int row = mt * 16 + gq + 8 * hr;
       if (row >= M) continue;
-      const int owner = row / rows_per, lr = row - owner * rows_per;
-      float* dst = cl.map_shared_rank(recv, owner) + ((size_t)rank * rows_per + lr) * r;
 #pragma unroll
       for (int n = 0; n < 2; ++n) {
         const int col = (2 * np + n) * 8 + 2 * tq;
-        *reinterpret_cast<float2*>(dst + col) = make_float2(acc[a][n][2 * hr], acc[a][n][2 * hr + 1]);
+        *reinterpret_cast<float2*>(tr + (size_t)row * r + col) = make_float2(acc[a][n][2 * hr], acc[a][n][2 * hr + 1]);
       }
     }
-  }
-  cl.sync();
-  const int r0 = rank * rows_per, nr = max(0, min(rows_per, M - r0));
-  for (int e = tid; e < nr * r; e += 256) {
-    float sum = 0.f;
-#pragma unroll
-    for (int c = 0; c < TK_CL; ++c) sum += recv[(size_t)c * rows_per * r + e];
-    t[(size_t)r0 * r + e] = sum;
   }
   RDL_TRACE_POINT(0, 4);
 }
@@ -351,10 +337,24 @@ __global__ void __launch_bounds__(SC_WARPS * 32, 1)
   grid_dep_launch();
   RDL_TRACE_POINT(1, 1);
   if (r > 0) {
+    // t rows = the TK_CL partials of dec_t_kernel summed in rank order
     const int nu = r / 4;                       // 16-byte units per t row
+    const size_t pstride = (size_t)gridDim.z * Lq * r;
     for (int e = tid; e < Lq * nu; e += NT) {
       const int i = e / nu, u = e % nu;
-      cp_async16(smem_u32(ts + i * (r + 8) + u * 4), t + (size_t)(b * Lq + i) * r + u * 4);
+      const float4* src = reinterpret_cast<const float4*>(t + (size_t)(b * Lq + i) * r + u * 4);
+      float4 pv[TK_CL];
+#pragma unroll
+      for (int k = 0; k < TK_CL; ++k) pv[k] = __ldcg(src + k * (pstride / 4));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < TK_CL; ++k) {
+        acc.x += pv[k].x;
+        acc.y += pv[k].y;
+        acc.z += pv[k].z;
+        acc.w += pv[k].w;
+      }
+      *reinterpret_cast<float4*>(ts + i * (r + 8) + u * 4) = acc;
     }
   }
   cp_async_commit();
@@ -619,6 +619,12 @@ __global__ void __launch_bounds__(DK_THREADS) dec_topk_kernel(const float* __res
   __shared__ int ncand_s;
   __shared__ __align__(8) uint64_t zbar;
   RDL_TRACE_POINT(2, 0);
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // the row position is an input of the call (read before the wait: this kernel starts
+  // early only behind the scorer, which has waited)
+  const int p = q_pos ? __ldcg(q_pos + (size_t)b * Lq + i) : i;
   if (threadIdx.x == 0) {
     tc::mbar_init(&zbar, 1);
     tc::mbar_fence_init();
@@ -627,14 +633,10 @@ __global__ void __launch_bounds__(DK_THREADS) dec_topk_kernel(const float* __res
   grid_dep_wait();
   grid_dep_launch();
   RDL_TRACE_POINT(2, 1);
-  const int C = L / S, G = Hq / Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   uint32_t* keys = dk_smem;                                        // [C]
   float* zs = reinterpret_cast<float*>(dk_smem + ((C + 3) & ~3));  // [G][C] (ZS)
   const float* z0 = z_all + ((size_t)(b * Hq + g * G) * Lq + i) * C;
   const size_t hstride = (size_t)Lq * C;
-  const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
   int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
   if (is_mask_slot(p)) {
     for (int e = tid; e < K * G; e += DK_THREADS) {
@@ -771,7 +773,7 @@ constexpr int AT_THREADS = (AT_CONS + 1) * 32;
 constexpr int AT_STAGE_BYTES = 32768;
 constexpr int AT_MAXC = 2048;            // chunks per sequence on this path
 constexpr int AT_QROWS = 32;             // query rows per sequence on this path
-constexpr int AT_SLAB_WORK = 1;          // partition weight of one slab load, in row pairs
+constexpr int AT_SLAB_WORK = 2;          // partition weight of one slab load, in row pairs
 
 // window slabs a row at position p touches: [wlo(p), whi(p)] (w >= 0)
 __device__ __forceinline__ int win_lo(int p, int w) { return max(0, p - w) / S; }
@@ -826,6 +828,40 @@ __device__ __forceinline__ int cta_excl_scan(int v, int* ws, int& total) {
   return basev + x - v;
 }
 
+// Exclusive scan of two ints per thread over the whole CTA (blockDim.x <= 1024); returns the
+// thread's two exclusive prefixes and the two CTA totals.  ws: 2 * blockDim.x / 32 ints.
+__device__ __forceinline__ int2 cta_excl_scan2(int a, int bv, int* ws, int& ta, int& tb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = a, y = bv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, x, o), ya = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) {
+      x += xa;
+      y += ya;
+    }
+  }
+  if (lane == 31) {
+    ws[2 * warp] = x;
+    ws[2 * warp + 1] = y;
+  }
+  __syncthreads();
+  int ba = 0, bb = 0, sa = 0, sb = 0;
+  for (int w8 = 0; w8 < nw; ++w8) {
+    const int va = ws[2 * w8], vb = ws[2 * w8 + 1];
+    if (w8 < warp) {
+      ba += va;
+      bb += vb;
+    }
+    sa += va;
+    sb += vb;
+  }
+  __syncthreads();
+  ta = sa;
+  tb = sb;
+  return make_int2(ba + x - a, bb + y - bv);
+}
+
 // task word: row (6 bits) << 8 | kind (window = 128) | slot (7 bits)
 constexpr int TASK_WIN = 128;
 
@@ -871,11 +907,34 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     misc[1] = -1;
     misc[2] = 0;
   }
+  // ---------------- prologue: inputs of the call only (this kernel starts early only behind
+  // a kernel that has itself waited for its predecessor): positions, the query rows (waited
+  // for with the idx rows) and the window tasks per slab
+  for (int e = tid; e < Lq; e += AT_THREADS) pos_s[e] = q_pos ? __ldcg(q_pos + (size_t)b * Lq + e) : e;
+  for (int e = tid; e < Lq * 8 * 16 && tid < AT_CONS * 32; e += AT_CONS * 32) {   // consumer threads only
+    const int i = e >> 7, hd = (e >> 4) & 7, u = e & 15;
+    unsigned char* dst = qs + i * 2048 + hd * 256 + ((u ^ hd) << 4);
+    if (hd < G)
+      cp_async16(smem_u32(dst), q + ((size_t)(b * Lq + i) * Hq + g * G + hd) * D + u * 8);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();                      // group 1: query rows
+  for (int c = tid; c < C; c += AT_THREADS) hist[c] = 0;
+  __syncthreads();
+  if (w >= 0) {
+    for (int i = warp; i < Lq; i += AT_CONS + 1) {
+      const int p = pos_s[i];
+      if (ROUTE && is_mask_slot(p)) continue;
+      const int lo = win_lo(p, w), hi = win_hi(p, w, L);
+      for (int t = lo + lane; t <= hi; t += 32) atomicAdd(&hist[t], 1);
+    }
+  }
   grid_dep_wait();
   grid_dep_launch();
   RDL_TRACE_POINT(3, 1);
 
-  // ---------------- one load batch: idx rows of the group, positions, query rows
+  // ---------------- idx rows of the group
   const int nent = Lq * Kt;
   const int32_t* ib = ROUTE ? idx + (size_t)(b * Hkv + g) * Lq * K : nullptr;
   if (ROUTE) {
@@ -885,22 +944,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (int e = tid; e < nent; e += AT_THREADS) idx_s[e] = ib[e];
     }
   }
-  for (int e = tid; e < Lq; e += AT_THREADS) pos_s[e] = q_pos ? q_pos[(size_t)b * Lq + e] : e;
-  cp_async_commit();                      // group 1: idx; group 2: the query rows (waited for later)
-  for (int e = tid; e < Lq * 8 * 16 && tid < AT_CONS * 32; e += AT_CONS * 32) {   // consumer threads only
-    const int i = e >> 7, hd = (e >> 4) & 7, u = e & 15;
-    unsigned char* dst = qs + i * 2048 + hd * 256 + ((u ^ hd) << 4);
-    if (hd < G)
-      cp_async16(smem_u32(dst), q + ((size_t)(b * Lq + i) * Hq + g * G + hd) * D + u * 8);
-    else
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  cp_async_commit();
-  for (int c = tid; c < C; c += AT_THREADS) hist[c] = 0;
-  cp_async_wait<1>();
+  cp_async_commit();                      // group 2: idx
+  cp_async_wait<0>();
   __syncthreads();
   RDL_TRACE_POINT(3, 4);
-  // ---------------- tasks per slab (the same on every CTA of the group)
+  // ---------------- chunk tasks per slab (the same on every CTA of the group)
   auto chunk_ok = [&](int e, int c) -> bool {   // entry e of idx_s holds chunk c >= 0
     if (c >= C) return false;
     if (flags & RDL_FLAG_CHECKS) return chunk_eligible(c, pos_s[e / K], w);
@@ -917,40 +965,36 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       atomicAdd(&hist[c], 1);
     }
   }
-  if (w >= 0) {
-    for (int i = warp; i < Lq; i += AT_CONS + 1) {
-      const int p = pos_s[i];
-      if (ROUTE && is_mask_slot(p)) continue;
-      const int lo = win_lo(p, w), hi = win_hi(p, w, L);
-      for (int t = lo + lane; t <= hi; t += 32) atomicAdd(&hist[t], 1);
-    }
-  }
   __syncthreads();
-  // work of slab c: its row pairs plus one slab load (weighted AT_SLAB_WORK pairs; heavier
-  // weights measured slower: the pairs of a slab every row selected dominate);
-  // exclusive prefix in chunk order.
-  // Slab c belongs to CTA floor(prefix(c) * R / total): contiguous slab ranges of equal work.
-  int* scan_ws = misc + 32;                                  // 9 ints
-  const int seg = (C + AT_THREADS - 1) / AT_THREADS;
-  const int s0 = min(C, tid * seg), s1 = min(C, s0 + seg);
+  // One scan gives both prefixes in chunk order: pre[c] = first list position of slab c's
+  // tasks, and the work prefix, work of slab c = its row pairs plus one slab load (weighted
+  // AT_SLAB_WORK pairs).  Slab c belongs to CTA floor(work prefix(c) * R / total work):
+  // contiguous slab ranges of equal work.
+  int* scan_ws = misc + 32;                                  // 32 ints
   {
-    int local = 0;
+    const int seg = (C + AT_THREADS - 1) / AT_THREADS;
+    const int s0 = min(C, tid * seg), s1 = min(C, s0 + seg);
+    int lt = 0, lw = 0;
     for (int c = s0; c < s1; ++c) {
       const int n = hist[c];
-      local += n > 0 ? (n + 1) / 2 + AT_SLAB_WORK : 0;
+      lt += n;
+      lw += n > 0 ? (n + 1) / 2 + AT_SLAB_WORK : 0;
     }
-    int total;
-    int run = cta_excl_scan(local, scan_ws, total);
-    // run * R < 2^31: at most C slabs x (Lq/2 + K + AT_SLAB_WORK) units x 148 CTAs
+    int tot_t, tot_w;
+    const int2 pr = cta_excl_scan2(lt, lw, scan_ws, tot_t, tot_w);
+    int rt = pr.x, rw = pr.y;
+    // rw * R < 2^31: at most C slabs x (Lq/2 + K + AT_SLAB_WORK) units x 148 CTAs
     for (int c = s0; c < s1; ++c) {
       const int n = hist[c];
+      pre[c] = rt;
+      rt += n;
       if (n > 0) {
-        const int owner = (run * R) / total;
+        const int owner = (rw * R) / tot_w;
         if (owner == j) {
           atomicMin(&misc[0], c);
           atomicMax(&misc[1], c);
         }
-        run += (n + 1) / 2 + AT_SLAB_WORK;
+        rw += (n + 1) / 2 + AT_SLAB_WORK;
       }
     }
   }
@@ -987,30 +1031,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   }
 
   // ---------------- consumer warps only from here (named barrier 1, AT_CONS warps)
-  // task cursors: pre[c] = first list position of slab c (prefix of the task counts)
-  {
-    constexpr int NCT = AT_CONS * 32;
-    const int cseg = (C + NCT - 1) / NCT;
-    const int q0 = min(C, tid * cseg), q1 = min(C, q0 + cseg);
-    int local = 0;
-    for (int c = q0; c < q1; ++c) local += hist[c];
-    int x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scan_ws[warp] = x;
-    asm volatile("bar.sync 1, %0;\n" ::"n"(NCT) : "memory");
-    int run = 0;
-    for (int w8 = 0; w8 < warp; ++w8) run += scan_ws[w8];
-    run += x - local;
-    for (int c = q0; c < q1; ++c) {
-      pre[c] = run;
-      run += hist[c];
-    }
-    asm volatile("bar.sync 1, %0;\n" ::"n"(NCT) : "memory");
-  }
   const int lbase = c_lo < c_hi ? pre[c_lo] : 0;   // list positions relative to this CTA
   const int lcap = Lq * (Kt + nwt);
   asm volatile("bar.sync 1, %0;\n" ::"n"(AT_CONS * 32) : "memory");
