@@ -108,9 +108,8 @@ bool dec_attn_rows_ok(const rdl_dims* dm, rdl_dtype t) {
 bool dec_attn_ok(const rdl_dims* dm, rdl_dtype t) { return dec_attn_rows_ok(dm, t) && dm->K <= kMaxK; }
 bool dec_swa_ok(const rdl_dims* dm, rdl_dtype t) { return dec_attn_rows_ok(dm, t) && dm->w >= 0; }
 int dec_attn_stages(const rdl_dims* dm, int K) {
-  const int nwt = dec::max_win_slabs(dm->w);
   for (int st = 4; st >= 2; --st)
-    if (dec::attn_smem(st, dm->Lq, K, dm->L / S, nwt).total <= 232448) return st;
+    if (dec::attn_smem(st, dm->Lq, K, dm->L / S).total <= 232448) return st;
   return 0;
 }
 int dec_attn_ranges(const rdl_dims* dm) {
@@ -205,14 +204,13 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
   AttnWs w{};
   if (!fast_attn(dm, t)) return w;
   if (dec_attn_ok(dm, t) && dec_attn_stages(dm, dm->K) > 0) {
-    // chunk outputs [B, Lq, Hkv, K, G, d], window slab sums [B, Lq, Hkv, nwt, G, d] and
-    // their (max, sum) [B, Lq, Hkv, nwt, G]
+    // chunk outputs [B, Lq, Hkv, K, G, d], the window part's unnormalised vector
+    // [B, Lq, Hq, d] and its (max, sum) [B, Lq, Hq]
     const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
-    const size_t nwt = (size_t)dec::max_win_slabs(dm->w);
     size_t off = 0;
     w.o_acc = off;   off += align256(sizeof(float) * rows * dm->K * dm->d);
-    w.o_loc = off;   off += align256(sizeof(float) * rows * nwt * dm->d);
-    w.lam_loc = off; off += align256(sizeof(float2) * rows * nwt);
+    w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d);
+    w.lam_loc = off; off += align256(sizeof(float2) * rows);
     w.total = off;
     return w;
   }
@@ -340,13 +338,26 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
   const AttnWs wl = attn_ws(dm, RDL_BF16);
   char* ws = static_cast<char*>(workspace);
   float* o_part = reinterpret_cast<float*>(ws + wl.o_acc);
-  float* ow_part = reinterpret_cast<float*>(ws + wl.o_loc);
-  float2* ml_part = reinterpret_cast<float2*>(ws + wl.lam_loc);
+  float* ow = reinterpret_cast<float*>(ws + wl.o_loc);
+  float2* ml = reinterpret_cast<float2*>(ws + wl.lam_loc);
   const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
   CUtensorMap kmap, vmap;
   if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
   const int stages = dec_attn_stages(dm, dm->K);
-  const int smem = dec::attn_smem(stages, dm->Lq, dm->K, dm->L / S, dec::max_win_slabs(dm->w)).total;
+  const int smem = dec::attn_smem(stages, dm->Lq, dm->K, dm->L / S).total;
+  const float sl2w = (float)(1.0 / sqrt((double)dm->d) * 1.4426950408889634);
+  if (dm->w >= 0) {
+    // the local window, while the top-K of the step may still run (reads inputs only)
+    const int wsm = dec::swa_smem();
+    if (cudaFuncSetAttribute(dec::dec_swa_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, wsm) !=
+        cudaSuccess)
+      return RDL_ERR_CUDA;
+    const int ctas = dm->B * dm->Hkv * ((dm->Lq + 1) / 2);
+    if (launch_pdl(dec::dec_swa_kernel<true>, dim3(ctas), dim3(dec::SW_WARPS * 32), wsm, st, kmap, vmap,
+                   static_cast<const __nv_bfloat16*>(q), q_pos, dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->w, sl2w,
+                   (__nv_bfloat16*)nullptr, (float*)nullptr, ow, ml) != cudaSuccess)
+      return RDL_ERR_CUDA;
+  }
   auto kern = dec::dec_attn_kernel<true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return RDL_ERR_CUDA;
@@ -355,11 +366,18 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
   if (launch_pdl(kern, dim3(dm->B * dm->Hkv * R), dim3(dec::AT_THREADS), smem, st, kmap, vmap,
                  static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
                  static_cast<const __nv_bfloat16*>(q), q_pos, idx, dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->K, dm->w,
-                 dm->flags, R, stages, sl2, o_part, ow_part, ml_part) != cudaSuccess)
+                 dm->flags, R, stages, sl2, o_part) != cudaSuccess)
     return RDL_ERR_CUDA;
   const long long items = (long long)dm->B * dm->Lq * dm->Hq;
-  if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, st, q_pos, idx, z_sel,
-                 (const float*)o_part, (const float*)ow_part, (const float2*)ml_part, dm->B, dm->L, dm->Lq, dm->Hq,
+  // The combine is launched early; its shared-memory request keeps it at one CTA per SM, so
+  // its CTAs spread over the SMs as the attention CTAs retire instead of piling onto the
+  // first free ones (measured 6 CTAs per SM and twice the time otherwise).
+  if (cudaFuncSetAttribute(dec::dec_comb_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dec::COMB_SPREAD_SMEM) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), dec::COMB_SPREAD_SMEM, st,
+                 q_pos, idx, z_sel,
+                 (const float*)o_part, (const float*)ow, (const float2*)ml, dm->B, dm->L, dm->Lq, dm->Hq,
                  dm->Hkv, dm->K, dm->w, dm->flags, static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
     return RDL_ERR_CUDA;
   return RDL_OK;
@@ -702,13 +720,14 @@ rdl_status rdl_swa_attn(const void* q, const int32_t* q_pos, const void* k, cons
     CUtensorMap kmap, vmap;
     if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows)) return RDL_ERR_CUDA;
     const int smem = dec::swa_smem();
-    if (cudaFuncSetAttribute(dec::dec_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(dec::dec_swa_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
       return RDL_ERR_CUDA;
     const float sl2 = (float)(1.0 / sqrt((double)dims->d) * 1.4426950408889634);
     const int ctas = dims->B * dims->Hkv * ((dims->Lq + 1) / 2);
-    if (launch_pdl(dec::dec_swa_kernel, dim3(ctas), dim3(dec::SW_WARPS * 32), smem, st, kmap, vmap,
+    if (launch_pdl(dec::dec_swa_kernel<false>, dim3(ctas), dim3(dec::SW_WARPS * 32), smem, st, kmap, vmap,
                    static_cast<const __nv_bfloat16*>(q), q_pos, dims->L, dims->Lq, dims->Hq, dims->Hkv, dims->w, sl2,
-                   static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
+                   static_cast<__nv_bfloat16*>(o), lse, (float*)nullptr, (float2*)nullptr) != cudaSuccess)
       return RDL_ERR_CUDA;
     return RDL_OK;
   }

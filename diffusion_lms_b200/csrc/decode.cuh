@@ -755,18 +755,16 @@ __global__ void __launch_bounds__(DK_THREADS) dec_topk_kernel(const float* __res
 // =====================================================================================
 // dec_attn_kernel: chunk-major two-level attention for decode blocks.
 //
-// Work items: for KV group (b, g), every 64-key slab c that some row needs -- because the
-// row selected chunk c (a chunk task: second-level softmax over the 63 content keys) or
-// because slab c overlaps the row's window (a window task: the window keys of that slab).
-// The R CTAs of a group all build the same histogram of tasks per slab from idx and the
-// row positions and split the prefix of (row pairs + one slab load) into R equal shares,
-// so a chunk that every row selected costs one CTA as much as many sparse ones.  A CTA
-// streams its slabs once through a TMA ring; each consumer warp computes two tasks of a
-// slab at once (M = 16 = two rows x 8 head slots) with the probabilities kept in
-// registers (no shared-memory round trip), and writes one partial per task:
-//   chunk task  -> o_part[b,i,g,k]  = softmax-normalised output of chunk idx[k]
-//   window task -> ow_part[b,i,g,s] = unnormalised sum, ml_part = (max, sum) of slab s
-// dec_comb_kernel merges the partials of a row in a fixed order.
+// Work items: for KV group (b, g), every selected chunk c, with one task per row that
+// selected it (second-level softmax over its 63 content keys); the local window is
+// computed by dec_swa_kernel<true> while the top-K still runs.  The R CTAs of a group all
+// build the same histogram of tasks per chunk from idx and split the prefix of (row pairs
+// + one slab load) into R equal shares, so a chunk that every row selected costs one CTA
+// as much as many sparse ones.  A CTA streams its chunks' K/V once through a TMA ring;
+// each consumer warp computes two tasks of a slab at once (M = 16 = two rows x 8 head
+// slots) with the probabilities kept in registers (no shared-memory round trip), and
+// writes o_part[b,i,g,k] = the softmax-normalised output of chunk idx[k].
+// dec_comb_kernel merges a row's window part and chunk outputs in a fixed order.
 // =====================================================================================
 constexpr int AT_CONS = 15;
 constexpr int AT_THREADS = (AT_CONS + 1) * 32;
@@ -784,7 +782,7 @@ __host__ __device__ inline int max_win_slabs(int w) { return w < 0 ? 0 : (2 * w)
 struct AttnSmem {
   int ring, qs, idx, pos, hist, pre, list, bar, misc, total;
 };
-__host__ __device__ inline AttnSmem attn_smem(int stages, int Lq, int K, int C, int nwt) {
+__host__ __device__ inline AttnSmem attn_smem(int stages, int Lq, int K, int C) {
   AttnSmem s{};
   int off = 0;
   s.ring = off; off += stages * AT_STAGE_BYTES;
@@ -793,7 +791,7 @@ __host__ __device__ inline AttnSmem attn_smem(int stages, int Lq, int K, int C, 
   s.pos = off;  off += ((Lq + 3) & ~3) * 4;
   s.hist = off; off += ((C + 3) & ~3) * 4;
   s.pre = off;  off += ((C + 3) & ~3) * 4;
-  s.list = off; off += ((Lq * (K + nwt) + 3) & ~3) * 4;
+  s.list = off; off += ((Lq * K + 3) & ~3) * 4;
   s.bar = off;  off += 16 * stages;
   s.misc = off; off += 256;
   s.total = off + 1024;
@@ -862,8 +860,7 @@ __device__ __forceinline__ int2 cta_excl_scan2(int a, int bv, int* ws, int& ta, 
   return make_int2(ba + x - a, bb + y - bv);
 }
 
-// task word: row (6 bits) << 8 | kind (window = 128) | slot (7 bits)
-constexpr int TASK_WIN = 128;
+// task word: row << 8 | slot (slot < 128)
 
 template <bool ROUTE>
 __global__ void __launch_bounds__(AT_THREADS, 1)
@@ -871,15 +868,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     const __nv_bfloat16* __restrict__ kv_base_k, const __nv_bfloat16* __restrict__ kv_base_v,
                     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
                     const int32_t* __restrict__ idx, int L, int Lq, int Hq, int Hkv, int K, int w, int flags,
-                    int R, int stages, float sl2, float* __restrict__ o_part, float* __restrict__ ow_part,
-                    float2* __restrict__ ml_part) {
+                    int R, int stages, float sl2, float* __restrict__ o_part) {
   constexpr int D = 128;
   extern __shared__ unsigned char at_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(at_raw) + 1023) & ~uintptr_t(1023));
   const int C = L / S, G = Hq / Hkv;
-  const int nwt = max_win_slabs(w);
   const int Kt = ROUTE ? K : 0;
-  const AttnSmem SL = attn_smem(stages, Lq, Kt, C, nwt);
+  const AttnSmem SL = attn_smem(stages, Lq, Kt, C);
   unsigned char* ring = base + SL.ring;
   unsigned char* qs = base + SL.qs;
   int* idx_s = reinterpret_cast<int*>(base + SL.idx);
@@ -907,9 +902,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     misc[1] = -1;
     misc[2] = 0;
   }
-  // ---------------- prologue: inputs of the call only (this kernel starts early only behind
-  // a kernel that has itself waited for its predecessor): positions, the query rows (waited
-  // for with the idx rows) and the window tasks per slab
+  // ---------------- prologue: inputs of the call only (this kernel starts early only when
+  // every kernel before the call has completed): positions and the query rows (waited for
+  // with the idx rows)
   for (int e = tid; e < Lq; e += AT_THREADS) pos_s[e] = q_pos ? __ldcg(q_pos + (size_t)b * Lq + e) : e;
   for (int e = tid; e < Lq * 8 * 16 && tid < AT_CONS * 32; e += AT_CONS * 32) {   // consumer threads only
     const int i = e >> 7, hd = (e >> 4) & 7, u = e & 15;
@@ -921,15 +916,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   }
   cp_async_commit();                      // group 1: query rows
   for (int c = tid; c < C; c += AT_THREADS) hist[c] = 0;
-  __syncthreads();
-  if (w >= 0) {
-    for (int i = warp; i < Lq; i += AT_CONS + 1) {
-      const int p = pos_s[i];
-      if (ROUTE && is_mask_slot(p)) continue;
-      const int lo = win_lo(p, w), hi = win_hi(p, w, L);
-      for (int t = lo + lane; t <= hi; t += 32) atomicAdd(&hist[t], 1);
-    }
-  }
   grid_dep_wait();
   grid_dep_launch();
   RDL_TRACE_POINT(3, 1);
@@ -1032,7 +1018,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
   // ---------------- consumer warps only from here (named barrier 1, AT_CONS warps)
   const int lbase = c_lo < c_hi ? pre[c_lo] : 0;   // list positions relative to this CTA
-  const int lcap = Lq * (Kt + nwt);
+  const int lcap = Lq * Kt;
   asm volatile("bar.sync 1, %0;\n" ::"n"(AT_CONS * 32) : "memory");
   if (ROUTE && c_lo < c_hi) {
     for (int e = tid; e < nent; e += AT_CONS * 32) {
@@ -1041,18 +1027,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const int slot = atomicAdd(&pre[c], 1) - lbase;
       if (slot < lcap) list[slot] = ((e / K) << 8) | (e % K);
       else record_status(RDL_ERR_DEVICE_CHECK);
-    }
-  }
-  if (w >= 0 && c_lo < c_hi) {
-    for (int i = warp; i < Lq; i += AT_CONS) {
-      const int p = pos_s[i];
-      if (ROUTE && is_mask_slot(p)) continue;
-      const int lo = win_lo(p, w), hi = min(win_hi(p, w, L), c_hi - 1);
-      for (int t = max(lo, c_lo) + lane; t <= hi; t += 32) {
-        const int slot = atomicAdd(&pre[t], 1) - lbase;
-        if (slot < lcap) list[slot] = (i << 8) | TASK_WIN | (t - lo);
-        else record_status(RDL_ERR_DEVICE_CHECK);
-      }
     }
   }
   RDL_TRACE_POINT(3, 2);
@@ -1101,21 +1075,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           }
         }
       }
-      // ---- per-row mask and softmax (row gq: task A, row gq + 8: task B)
-      const bool winA = (tA & TASK_WIN) != 0, winB = (tB & TASK_WIN) != 0;
-      const int pA = pos_s[iA], pB = pos_s[iB];
+      // ---- softmax over the chunk's content keys (row gq: task A, row gq + 8: task B)
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int key = 8 * nt + 2 * tq + (e & 1);
-          const bool hb = e >= 2;
-          const bool win = hb ? winB : winA;
-          const int p = hb ? pB : pA;
-          const int j2 = S * c + key;
-          const bool in = win ? (j2 >= p - w && j2 <= p + w) : key < CONTENT;
-          const float v = in ? sc[nt][e] * sl2 : -INFINITY;
+          const int hb = e >> 1;
+          const float v = key < CONTENT ? sc[nt][e] * sl2 : -INFINITY;
           sc[nt][e] = v;
           mx[hb] = fmaxf(mx[hb], v);
         }
@@ -1139,8 +1107,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 1);
         sm[hb] += __shfl_xor_sync(0xffffffffu, sm[hb], 2);
       }
-      // chunk tasks are normalised here; window tasks keep (max, sum) for the merge
-      const float fA = winA ? 1.f : 1.f / sm[0], fB = winB ? 1.f : 1.f / sm[1];
+      const float fA = 1.f / sm[0], fB = 1.f / sm[1];
       // P as bf16 A fragments (FA2 layout: the S accumulators of n-tiles 2kk, 2kk+1)
       uint32_t pa[4][4];
 #pragma unroll
@@ -1156,11 +1123,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const int slotA = tA & 127, slotB = tB & 127;
         const size_t rgA = (size_t)(b * Lq + iA) * Hkv + g, rgB = (size_t)(b * Lq + iB) * Hkv + g;
         if (gq < G) {
-          dstA = (tA & TASK_WIN) ? ow_part + ((rgA * nwt + slotA) * G + gq) * D : o_part + ((rgA * K + slotA) * G + gq) * D;
-          if (hasB)
-            dstB = (tB & TASK_WIN) ? ow_part + ((rgB * nwt + slotB) * G + gq) * D : o_part + ((rgB * K + slotB) * G + gq) * D;
-          if (tq == 0 && (tA & TASK_WIN)) ml_part[(rgA * nwt + slotA) * G + gq] = make_float2(mx[0] * LN2, sm[0]);
-          if (tq == 0 && hasB && (tB & TASK_WIN)) ml_part[(rgB * nwt + slotB) * G + gq] = make_float2(mx[1] * LN2, sm[1]);
+          dstA = o_part + ((rgA * K + slotA) * G + gq) * D;
+          if (hasB) dstB = o_part + ((rgB * K + slotB) * G + gq) * D;
         }
       }
       // ---- O = P V, 64 dims at a time
@@ -1208,15 +1172,22 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 // CTA = (b, g, pair of query rows); warp w streams window slabs w, w + SW_WARPS, ... of the
 // pair through its own shared-memory slot (TMA), keeps an online softmax per row (M = 16 =
 // two rows x 8 head slots), and the warps' partial states are merged in a fixed order.
+// ROUTE_WIN: the local-window part of a route layer.  It reads only inputs of the call, so
+// it runs while the top-K of the same step is still running: it releases its dependent at
+// once and waits for its own predecessor only before it exits (its completion then implies
+// the predecessor's).  It writes the window's (max, sum) and unnormalised vector per
+// (row, head) for dec_comb_kernel instead of the normalised output.
 // =====================================================================================
 constexpr int SW_WARPS = 6;
 
 __host__ __device__ inline int swa_smem() { return 1024 + SW_WARPS * AT_STAGE_BYTES + 2 * 2048 + 64 * SW_WARPS; }
 
+template <bool ROUTE_WIN>
 __global__ void __launch_bounds__(SW_WARPS * 32, 1)
     dec_swa_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos, int L, int Lq, int Hq,
-                   int Hkv, int w, float sl2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+                   int Hkv, int w, float sl2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                   float* __restrict__ ow, float2* __restrict__ ml) {
   constexpr int D = 128;
   extern __shared__ unsigned char sw_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sw_raw) + 1023) & ~uintptr_t(1023));
@@ -1234,8 +1205,9 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
     for (int x = 0; x < SW_WARPS; ++x) tc::mbar_init(&bar[x], 1);
     tc::mbar_fence_init();
   }
-  grid_dep_wait();
+  if (!ROUTE_WIN) grid_dep_wait();
   grid_dep_launch();
+  RDL_TRACE_POINT(5, 0);
   const int pA = q_pos ? q_pos[(size_t)b * Lq + iA] : iA;
   const int pB = q_pos ? q_pos[(size_t)b * Lq + iB] : iB;
   // query rows of the pair: [row][8 heads][256 B], 16-byte units ^ head; head 7+ zero
@@ -1413,6 +1385,13 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
       for (int c = 0; c < 4; ++c) acc[c] += f * px[row * 128 + d4 + c];
     }
     const int i = hb ? iB : iA, h = g * G + hd;
+    if (ROUTE_WIN) {
+      // (max in natural-log units, sum) and the vector relative to that max
+      const size_t rh = (size_t)(b * Lq + i) * Hq + h;
+      *reinterpret_cast<float4*>(ow + rh * D + d4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      if (d4 == 0) ml[rh] = make_float2(Lsum > 0.f ? M * LN2 : -INFINITY, Lsum);
+      continue;
+    }
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     __nv_bfloat16* orow = o + ((size_t)(b * Lq + i) * Hq + h) * D + d4;
     const __nv_bfloat162 o01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
@@ -1423,22 +1402,26 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
     *reinterpret_cast<uint2*>(orow) = pk;
     if (lse && d4 == 0) lse[(size_t)(b * Hq + h) * Lq + i] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
   }
+  RDL_TRACE_POINT(5, 1);
+  if (ROUTE_WIN) grid_dep_wait();     // complete only after the predecessor (top-K) has
   (void)C;
 }
 
 // =====================================================================================
 // dec_comb_kernel: one warp per (b, i, h); lane l owns dims 4l .. 4l+3.  Merges the
-// window slab partials (max, sum, unnormalised vector) and, on route layers, the chunk
-// outputs with weights e^{z_c}: one partition, o = sum(weight * vector) / sum(weight).
-// Parts are loaded in batches before their weights are known (unused loads are harmless).
+// window part (max, sum, unnormalised vector) and, on route layers, the chunk outputs with
+// weights e^{z_c}: one partition, o = sum(weight * vector) / sum(weight), in a fixed order.
+// Chunk outputs are loaded in batches before their weights are known (unused loads are
+// harmless).
 // =====================================================================================
+constexpr int COMB_SPREAD_SMEM = 120 * 1024;   // dynamic shared memory requested (unused)
 template <bool ROUTE>
 __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict__ q_pos,
                                                        const int32_t* __restrict__ idx,
                                                        const float* __restrict__ z_sel,
                                                        const float* __restrict__ o_part,
-                                                       const float* __restrict__ ow_part,
-                                                       const float2* __restrict__ ml_part, int B, int L, int Lq,
+                                                       const float* __restrict__ ow,
+                                                       const float2* __restrict__ ml, int B, int L, int Lq,
                                                        int Hq, int Hkv, int K, int w, int flags,
                                                        __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
   constexpr int D = 128;
@@ -1454,27 +1437,21 @@ __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict
   const int C = L / S, G = Hq / Hkv, g = h / G, hl = h % G;
   const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
   if (ROUTE && is_mask_slot(p)) return;
-  const int nwt = max_win_slabs(w);
-  const int nw = w >= 0 ? win_hi(p, w, L) - win_lo(p, w) + 1 : 0;
+  const size_t rh = (size_t)(b * Lq + i) * Hq + h;
   const size_t rg = (size_t)(b * Lq + i) * Hkv + g;
-  // window slabs: lanes s, s + 32 hold slab s's (max, sum)
-  float wm[2] = {-INFINITY, -INFINITY}, wl[2] = {0.f, 0.f};
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int s2 = lane + 32 * u;
-    if (s2 < nw) {
-      const float2 ml = ml_part[(rg * nwt + s2) * G + hl];
-      wm[u] = ml.x;
-      wl[u] = ml.y;
-    }
+  // every load that does not depend on a weight is issued first: the window part (absent
+  // when w < 0 or the window is empty: sum 0), the chunk ids and logits (lanes k, k+32 hold
+  // slot k) and the first 16 chunk outputs
+  float2 wml = make_float2(-INFINITY, 0.f);
+  float4 vw = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (w >= 0) {
+    wml = ml[rh];
+    vw = *reinterpret_cast<const float4*>(ow + rh * D + 4 * lane);
   }
-  float4 vw[12];
-#pragma unroll
-  for (int s2 = 0; s2 < 12; ++s2)
-    vw[s2] = s2 < nw ? *reinterpret_cast<const float4*>(ow_part + ((rg * nwt + s2) * G + hl) * D + 4 * lane)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-  // chunk slots: lanes k, k+32 hold slot k's logit (-inf when empty or skipped)
-  float zk[2] = {-INFINITY, -INFINITY};
+  int ck[2] = {-1, -1};
+  float zr[2] = {-INFINITY, -INFINITY};
+  const float* pbase = o_part + (rg * K * G + hl) * D + 4 * lane;
+  float4 v0[16];
   if (ROUTE) {
     const int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
     const float* zrow = z_sel + ((size_t)(b * Hq + h) * Lq + i) * K;
@@ -1482,43 +1459,40 @@ __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict
     for (int u = 0; u < 2; ++u) {
       const int k = lane + 32 * u;
       if (k < K) {
-        const int c = irow[k];
-        bool ok = c >= 0 && c < C;
-        if (ok && (flags & RDL_FLAG_CHECKS) && !chunk_eligible(c, p, w)) ok = false;
-        if (ok) zk[u] = zrow[k];
+        ck[u] = irow[k];
+        zr[u] = zrow[k];
       }
     }
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      v0[u] = u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)u * G * D) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  float M = fmaxf(fmaxf(wl[0] > 0.f ? wm[0] : -INFINITY, wl[1] > 0.f ? wm[1] : -INFINITY), fmaxf(zk[0], zk[1]));
+  float zk[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int c = ck[u];
+    bool ok = ROUTE && c >= 0 && c < C;
+    if (ok && (flags & RDL_FLAG_CHECKS) && !chunk_eligible(c, p, w)) ok = false;
+    if (ok) zk[u] = zr[u];
+  }
+  const bool has_w = wml.y > 0.f;
+  float M = fmaxf(zk[0], zk[1]);
   M = warp_max(M);
+  if (has_w) M = fmaxf(M, wml.x);
   if (M == -INFINITY) M = 0.f;
-  const float ew0 = wl[0] > 0.f ? expf(wm[0] - M) : 0.f;     // slab weights e^{m - M}
-  const float ew1 = wl[1] > 0.f ? expf(wm[1] - M) : 0.f;
+  const float ew = has_w ? expf(wml.x - M) : 0.f;           // window weight e^{m - M}
   const float ek0 = zk[0] == -INFINITY ? 0.f : expf(zk[0] - M);
   const float ek1 = zk[1] == -INFINITY ? 0.f : expf(zk[1] - M);
-  const float Zs = warp_sum(ew0 * wl[0] + ew1 * wl[1] + ek0 + ek1);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int s2 = 0; s2 < 12; ++s2) {
-    const float f = __shfl_sync(0xffffffffu, ew0, s2);
-    if (s2 < nw && f != 0.f) {
-      acc.x += f * vw[s2].x; acc.y += f * vw[s2].y; acc.z += f * vw[s2].z; acc.w += f * vw[s2].w;
-    }
-  }
-  for (int s2 = 12; s2 < nw; ++s2) {
-    const float f = __shfl_sync(0xffffffffu, s2 < 32 ? ew0 : ew1, s2 & 31);
-    const float4 v = *reinterpret_cast<const float4*>(ow_part + ((rg * nwt + s2) * G + hl) * D + 4 * lane);
-    if (f != 0.f) {
-      acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
-    }
-  }
+  const float Zs = ew * wml.y + warp_sum(ek0 + ek1);
+  float4 acc = make_float4(ew * vw.x, ew * vw.y, ew * vw.z, ew * vw.w);
   if (ROUTE) {
-    const float* pbase = o_part + (rg * K * G + hl) * D + 4 * lane;
     for (int k0 = 0; k0 < K; k0 += 16) {
       float4 v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = k0 + u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)(k0 + u) * G * D)
-                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 16; ++u)
+        v[u] = k0 == 0 ? v0[u]
+                       : (k0 + u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)(k0 + u) * G * D)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f));
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int k = k0 + u;
