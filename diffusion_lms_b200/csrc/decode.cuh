@@ -954,8 +954,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __syncthreads();
   // One scan gives both prefixes in chunk order: pre[c] = first list position of slab c's
   // tasks, and the work prefix, work of slab c = its row pairs plus one slab load (weighted
-  // AT_SLAB_WORK pairs).  Slab c belongs to CTA floor(work prefix(c) * R / total work):
-  // contiguous slab ranges of equal work.
+  // AT_SLAB_WORK pairs).  Slab c belongs to CTA floor((work prefix(c) + work(c) / 2) * R /
+  // total work), the share that holds the slab's midpoint: contiguous slab ranges of equal
+  // work, a heavy slab overshooting a share by at most half its work.
   int* scan_ws = misc + 32;                                  // 32 ints
   {
     const int seg = (C + AT_THREADS - 1) / AT_THREADS;
@@ -975,12 +976,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       pre[c] = rt;
       rt += n;
       if (n > 0) {
-        const int owner = (rw * R) / tot_w;
+        const int wc = (n + 1) / 2 + AT_SLAB_WORK;
+        const int owner = min(R - 1, ((rw + wc / 2) * R) / tot_w);   // share holding the slab's midpoint
         if (owner == j) {
           atomicMin(&misc[0], c);
           atomicMax(&misc[1], c);
         }
-        rw += (n + 1) / 2 + AT_SLAB_WORK;
+        rw += wc;
       }
     }
   }
