@@ -33,6 +33,10 @@ METRIC = "route-layer sparse-attn query-tokens/s at 16K-128K; decode-step ms at 
 # DRAM bytes of one rdl_route_attn call on the 16K prefill (window + chunk kernels), from one
 # ncu capture of the current kernels; set to None when either kernel changes.
 ATTN_PREFILL_TRAFFIC = 934.6e6
+# DRAM bytes of one 128K decode step (the six decode kernels, one launch each, caches cold
+# between kernels under ncu, so intermediates re-read from DRAM here stay in L2 live); set to
+# None when a decode kernel changes.
+DECODE_STEP_TRAFFIC = 108.34e6
 UNIT = "query-tokens/s"
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -272,6 +276,10 @@ def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
             "query_tokens_per_s": world * 32 / (d_ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": d_ach / pk["hbm_gbs"], "algorithmic_bytes": db["total"],
+                         "traffic": DECODE_STEP_TRAFFIC,
+                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the six "
+                                           "decode kernels, one launch each "
+                                           "(profiles/launches_route_decode_128k.md)",
                          "unique_group_chunk_pairs": db["unique_pairs"],
                          "peak_source": f"hbm_gbs ({pk_kind})"}}
 
