@@ -16,6 +16,7 @@
 #include "chunk_attn.cuh"
 #include "tmap.cuh"
 #include "chunk_tc.cuh"
+#include "window_tc.cuh"
 #include "decode.cuh"
 #include <cstdlib>
 
@@ -522,6 +523,23 @@ rdl_status launch_window_mma(const void* q, const int32_t* q_pos, const void* k,
                              const rdl_dims* dm, void* o, float* lse, float* o_loc, float* lam_loc,
                              int nsplit, cudaStream_t st) {
   const int G = dm->Hq / dm->Hkv;
+  if (nsplit == 1 && dm->w >= 0 && G <= 8) {
+    // one key range per tile: the tcgen05 kernel (16 tokens x 8 head slots per CTA)
+    CUtensorMap qmap, kmap, vmap;
+    const unsigned long long tokens = (unsigned long long)dm->B * dm->Lq;
+    const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
+    if (!make_tmap_q_run(&qmap, q, tokens, (unsigned)dm->Hq, WT_TOK) ||
+        !make_tmap_kv_halves(&kmap, k, kvrows, WT_KEYS) || !make_tmap_kv_halves(&vmap, v, kvrows, WT_KEYS))
+      return RDL_ERR_CUDA;
+    auto tk = window_tc_kernel<MODE>;
+    if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, WT_SMEM) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    dim3 grid((dm->Lq + WT_TOK - 1) / WT_TOK, dm->B * dm->Hkv);
+    count_launch();
+    tk<<<grid, WT_THREADS, WT_SMEM, st>>>(qmap, kmap, vmap, q_pos, dm->L, dm->Lq, dm->Hq, dm->Hkv, dm->w,
+                                          static_cast<__nv_bfloat16*>(o), lse, o_loc, lam_loc);
+    return cuda_status(cudaGetLastError());
+  }
   const size_t smem = window_mma_smem(G);
   auto kern = window_mma_kernel<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -39,14 +39,15 @@ inline bool make_tmap_bf16(CUtensorMap* map, const void* base, unsigned long lon
 }
 
 // K or V of one KV head as [rows x 128] bf16 (row stride 256 B), viewed as (64 columns,
-// rows, 2 halves) so that one box of 64 rows x 2 halves lands as two 8 KB 128-byte-swizzled
-// tiles (columns 0-63, then 64-127).
-inline bool make_tmap_kv_halves(CUtensorMap* map, const void* base, unsigned long long rows) {
+// rows, 2 halves) so that one box of box_rows rows x 2 halves lands as two 128-byte-swizzled
+// tiles of box_rows x 128 B (columns 0-63, then 64-127).
+inline bool make_tmap_kv_halves(CUtensorMap* map, const void* base, unsigned long long rows,
+                                unsigned box_rows = 64) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {64, rows, 2};
   cuuint64_t strides[2] = {256, 128};
-  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t box[3] = {64, box_rows, 2};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
