@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 METRIC = "route-layer sparse-attn query-tokens/s at 16K-128K; decode-step ms at 128K"
 # DRAM bytes of one rdl_route_attn call on the 16K prefill (window + chunk kernels), from one
 # ncu capture of the current kernels; set to None when either kernel changes.
-ATTN_PREFILL_TRAFFIC = 934.6e6
+ATTN_PREFILL_TRAFFIC = 941.8e6
 # DRAM bytes of one 128K decode step (the six decode kernels, one launch each, caches cold
 # between kernels under ncu, so intermediates re-read from DRAM here stay in L2 live); set to
 # None when a decode kernel changes.
@@ -530,7 +530,7 @@ def main():
                 "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / pk["bf16_tflops"], "traffic": ATTN_PREFILL_TRAFFIC,
                 "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                  "window_mma_kernel<1> + chunk_tc_kernel, one launch each "
+                                  "window_tc_kernel<1> + chunk_tc_kernel, one launch each "
                                   "(profiles/attn_traffic_route_prefill_16k.md)",
                 "algorithmic_flops": fl_attn, "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
     elif dominant == "rdl_route_score_topk":
