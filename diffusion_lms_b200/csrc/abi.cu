@@ -17,6 +17,7 @@
 #include "tmap.cuh"
 #include "chunk_tc.cuh"
 #include "window_tc.cuh"
+#include "score_tc.cuh"
 #include "decode.cuh"
 #include <cstdlib>
 
@@ -414,7 +415,29 @@ rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const 
     kern<<<dim3((C + 31) / 32, dm->Hq, dm->B), 256, smem, st>>>(summary, static_cast<const __nv_bfloat16*>(w_up),
                                                                  C, dm->Hq, sb);
   }
-  {
+  if (dm->Hq / dm->Hkv <= 8) {
+    // tcgen05 scorer: q_h and the split chunk rows by TMA (views with 128-byte rows)
+    const unsigned long long tokens = (unsigned long long)M, srows = (unsigned long long)dm->B * dm->Hq * C;
+    CUtensorMap qmap, smap, spmap, tmap;
+    const cuuint64_t qd[4] = {64, tokens, 2, (cuuint64_t)dm->Hq}, qs[3] = {(cuuint64_t)dm->Hq * 256, 128, 256};
+    const cuuint32_t qb[4] = {64, ZT_ROWS, 2, 1};
+    const cuuint64_t sd[4] = {64, srows, 2, 2}, ss[3] = {768, 256, 128};          // [s_hi | s_lo | ..] rows
+    const cuuint32_t sbx[4] = {64, ZT_CH, 2, 2};
+    const cuuint64_t pd[3] = {64, srows, 2}, ps[2] = {768, 128};                  // [.. | s'_hi | s'_lo]
+    const cuuint32_t pb[3] = {64, ZT_CH, 2};
+    const cuuint64_t td[3] = {64, tokens, 2}, ts[2] = {256, 128};                 // [t_hi | t_lo] rows
+    const cuuint32_t tb[3] = {64, ZT_ROWS, 2};
+    if (!make_tmap_bf16_nd(&qmap, q, 4, qd, qs, qb) || !make_tmap_bf16_nd(&smap, sb, 4, sd, ss, sbx) ||
+        !make_tmap_bf16_nd(&spmap, reinterpret_cast<const char*>(sb) + 512, 3, pd, ps, pb) ||
+        !make_tmap_bf16_nd(&tmap, tt, 3, td, ts, tb))
+      return RDL_ERR_CUDA;
+    if (cudaFuncSetAttribute(zeta_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ZT_SMEM) != cudaSuccess)
+      return RDL_ERR_CUDA;
+    dim3 grid((C + ZT_CH - 1) / ZT_CH, (dm->Lq + ZT_ROWS - 1) / ZT_ROWS, dm->B * dm->Hkv);
+    count_launch();
+    zeta_tc_kernel<<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
+                                                      dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
+  } else {
     auto kern = zeta_mma_kernel<R>;
     const int smem = ZetaSmem<R>::TOTAL;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

@@ -54,6 +54,19 @@ inline bool make_tmap_kv_halves(CUtensorMap* map, const void* base, unsigned lon
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Any bf16 view with a 64-element (128-byte) innermost box dimension, 128-byte swizzle:
+// dims[0] = 64 columns, dims/strides (bytes) of the outer dimensions as given.  Outside the
+// tensor reads as zeros.
+inline bool make_tmap_bf16_nd(CUtensorMap* map, const void* base, unsigned nd, const cuuint64_t* dims,
+                              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nd, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Queries q [tokens, Hq, 128] bf16 viewed as (64 columns, Hq heads, 2 halves, tokens): one box
 // of 8 heads x 2 halves x R consecutive tokens lands token-major, 2 KB per token (half 0 of
 // its 8 head rows, then half 1), each 1 KB a 128-byte-swizzled tile.  Heads past Hq read as 0.
