@@ -68,6 +68,21 @@ def test_bf16_scattered_positions_ragged_rows():
     P.check_swa(wl, gpu, rows)
 
 
+def test_bf16_many_scattered_rows_partial_tiles():
+    """600 rows at scattered positions: enough tiles for the single-pass tensor-core window
+    and scorer kernels, with a partial 16-token window tile and partial 128-row score tiles."""
+    full = W.make_inputs(small(L=4096, Lq=4096, K=8, w=100), seed=21, n_needles=4)
+    rng = np.random.default_rng(7)
+    pos = np.sort(rng.choice(4096, size=600, replace=False))
+    wl = dataclasses.replace(full, dims=dataclasses.replace(full.dims, Lq=600),
+                             q=full.q[:, pos].copy(), x=full.x[:, pos].copy(),
+                             q_pos=pos.astype(np.int32)[None, :])
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(600)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(16, 2), (2, 2), (6, 1)])
 def test_group_sizes(Hq, Hkv):
     wl = W.make_inputs(small(L=1024, Lq=1024, Hq=Hq, Hkv=Hkv, K=6, w=70), seed=14, n_needles=2)
