@@ -19,7 +19,8 @@
 //   sprep_kernel     per (h, c): [s_hi | s_lo | s'_hi | s'_lo] bf16 rows (the B operand)
 //   zeta_mma_kernel  per (b, g, 128 query rows, 64 chunks): the split contraction for the
 //                    group's heads, entropy and eligibility, per-head scores to the
-//                    workspace and the group max zeta
+//                    workspace and the group max zeta (groups of more than 8 heads;
+//                    zeta_tc_kernel in score_tc.cuh runs the same contraction on tcgen05)
 #pragma once
 #include "common.cuh"
 

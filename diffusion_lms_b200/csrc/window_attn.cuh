@@ -5,7 +5,9 @@
 //
 // generic_attn_kernel: scalar fp32 kernel for any dtype / head dim, computing either the
 //   sliding-window output or the whole two-level route partition in one pass.
-// window_mma_kernel:   bf16, d = 128 banded flash kernel on mma.sync tensor cores.
+// window_mma_kernel:   bf16, d = 128 banded flash kernel on mma.sync tensor cores, used
+//   when the keys of a row tile are split over several CTAs (few query rows) or a group
+//   has more than 8 heads; otherwise window_tc.cuh runs the window on tcgen05.
 //   CTA = 16 consecutive query rows x one KV group; warp w = head w of the group, so the
 //   window's K/V tiles (64 keys, double-buffered via cp.async) are shared by every head.
 #pragma once
