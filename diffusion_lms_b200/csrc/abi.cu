@@ -415,7 +415,7 @@ rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const 
     kern<<<dim3((C + 31) / 32, dm->Hq, dm->B), 256, smem, st>>>(summary, static_cast<const __nv_bfloat16*>(w_up),
                                                                  C, dm->Hq, sb);
   }
-  if (dm->Hq / dm->Hkv <= 8) {
+  {
     // tcgen05 scorer: q_h and the split chunk rows by TMA (views with 128-byte rows)
     const unsigned long long tokens = (unsigned long long)M, srows = (unsigned long long)dm->B * dm->Hq * C;
     CUtensorMap qmap, smap, spmap, tmap;
@@ -437,15 +437,6 @@ rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const 
     count_launch();
     zeta_tc_kernel<<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
                                                       dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
-  } else {
-    auto kern = zeta_mma_kernel<R>;
-    const int smem = ZetaSmem<R>::TOTAL;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return RDL_ERR_CUDA;
-    dim3 grid((C + ZM_CH - 1) / ZM_CH, (dm->Lq + ZM_ROWS - 1) / ZM_ROWS, dm->B * dm->Hkv);
-    count_launch();
-    kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), q_pos, tt, sb, entropy, dm->Lq, dm->L,
-                                  dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
   }
   if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
   return launch_topk(zeta, z_all, q_pos, dm, idx, z_sel, st);

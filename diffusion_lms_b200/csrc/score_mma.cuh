@@ -12,15 +12,13 @@
 // product (error ~5e-4) is not enough.  Every fp32 operand is split into two bf16 terms,
 // a = a_hi + a_lo with |a - a_hi - a_lo| <= 2^-18 |a|, and the contraction is
 //     q.s_hi + q.s_lo + t_hi.s'_hi + t_hi.s'_lo + t_lo.s'_hi       (q is exact in bf16)
-// on mma.sync m16n8k16 with fp32 accumulation: ~1e-6 absolute score error.
+// on bf16 tensor cores with fp32 accumulation: ~1e-6 absolute score error.
 //
 // Kernels:
 //   xw_mma_kernel    t = x W_down on tensor cores, stored as [t_hi | t_lo] bf16
 //   sprep_kernel     per (h, c): [s_hi | s_lo | s'_hi | s'_lo] bf16 rows (the B operand)
-//   zeta_mma_kernel  per (b, g, 128 query rows, 64 chunks): the split contraction for the
-//                    group's heads, entropy and eligibility, per-head scores to the
-//                    workspace and the group max zeta (groups of more than 8 heads;
-//                    zeta_tc_kernel in score_tc.cuh runs the same contraction on tcgen05)
+// The contraction itself, with entropy, eligibility, the per-head scores and the group
+// maximum zeta, is zeta_tc_kernel (score_tc.cuh, tcgen05 tensor cores).
 #pragma once
 #include "common.cuh"
 
@@ -154,199 +152,6 @@ __global__ void __launch_bounds__(256) sprep_kernel(const float* __restrict__ su
       o[2 * D + R + m] = __float2bfloat16_rn(acc - __bfloat162float(hi));
     }
     __syncwarp();
-  }
-}
-
-// --------------------------------------------------------------------------- scores
-// CTA per (64-chunk tile, 128-row query tile, b*Hkv + g); 8 warps in a 4 x 2 grid, each
-// 32 rows x 32 chunks.  Per head: q_h tile + SB tile staged (double-buffered over heads).
-constexpr int ZM_ROWS = 128, ZM_CH = 64;
-
-template <int R>
-struct ZetaSmem {
-  static constexpr int SBW = 2 * 128 + 2 * R;               // bf16 per SB row
-  static constexpr int SB_ROWB = SBW * 2;                   // bytes
-  static constexpr int Q_BYTES = ZM_ROWS * 256;
-  static constexpr int SB_BYTES = ZM_CH * SB_ROWB;
-  static constexpr int STAGE = Q_BYTES + SB_BYTES;
-  static constexpr int TT_BYTES = ZM_ROWS * (4 * R);         // [t_hi | t_lo] rows
-  static constexpr int TOTAL = 2 * STAGE + TT_BYTES;
-};
-
-template <int R>
-__global__ void __launch_bounds__(256) zeta_mma_kernel(
-    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
-    const __nv_bfloat16* __restrict__ tt, const __nv_bfloat16* __restrict__ sb,
-    const float* __restrict__ entropy, int Lq, int L, int Hq, int Hkv, int w, float lambda,
-    float* __restrict__ z_all, float* __restrict__ zeta) {
-  using SM = ZetaSmem<R>;
-  constexpr int D = 128, SBW = SM::SBW, SB_ROWB = SM::SB_ROWB, TT_ROWB = 4 * R;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* TTs = smem_raw + 2 * SM::STAGE;
-  __shared__ float Hs[8][ZM_CH];
-  __shared__ int Ps[ZM_ROWS];
-
-  const int C = L / S, G = Hq / Hkv;
-  const int bg = blockIdx.z, b = bg / Hkv, g = bg % Hkv;
-  const int i0 = blockIdx.y * ZM_ROWS, c0 = blockIdx.x * ZM_CH;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wm = warp >> 1, wn = warp & 1;
-  const float tau = rsqrtf((float)D);
-
-  if (tid < ZM_ROWS) {
-    const int i = i0 + tid;
-    Ps[tid] = (i < Lq) ? (q_pos ? q_pos[(size_t)b * Lq + i] : i) : INT_MIN;
-  }
-  for (int e = tid; e < G * ZM_CH; e += 256) {
-    const int hl = e / ZM_CH, cc = e % ZM_CH, c = c0 + cc;
-    Hs[hl][cc] = (c < C) ? entropy[(size_t)(b * Hq + g * G + hl) * C + c] : 0.f;
-  }
-  // residual rows (shared by all heads)
-  for (int e = tid; e < ZM_ROWS * (TT_ROWB / 16); e += 256) {
-    const int r = e / (TT_ROWB / 16), ch = e % (TT_ROWB / 16);
-    const int i = min(i0 + r, Lq - 1);
-    cp_async16(smem_u32(TTs + swz(r, ch, TT_ROWB)), tt + ((size_t)b * Lq + i) * (2 * R) + ch * 8);
-  }
-  auto load_head = [&](int hl, int st) {
-    unsigned char* Qs = smem_raw + st * SM::STAGE;
-    unsigned char* Bs = Qs + SM::Q_BYTES;
-    const int h = g * G + hl;
-    for (int e = tid; e < ZM_ROWS * 16; e += 256) {
-      const int r = e >> 4, ch = e & 15;
-      const int i = min(i0 + r, Lq - 1);
-      cp_async16(smem_u32(Qs + swz(r, ch, 256)), q + ((size_t)(b * Lq + i) * Hq + h) * D + ch * 8);
-    }
-    for (int e = tid; e < ZM_CH * (SB_ROWB / 16); e += 256) {
-      const int r = e / (SB_ROWB / 16), ch = e % (SB_ROWB / 16);
-      const int c = min(c0 + r, C - 1);
-      cp_async16(smem_u32(Bs + swz(r, ch, SB_ROWB)), sb + ((size_t)(b * Hq + h) * C + c) * SBW + ch * 8);
-    }
-  };
-  load_head(0, 0);
-  cp_async_commit();
-
-  float zmax[2][4][4];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int n = 0; n < 4; ++n) zmax[a][n][0] = zmax[a][n][1] = zmax[a][n][2] = zmax[a][n][3] = -INFINITY;
-
-  const int gq = lane >> 2, tq = lane & 3;
-  for (int hl = 0; hl < G; ++hl) {
-    const int st = hl & 1;
-    if (hl + 1 < G) load_head(hl + 1, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const unsigned char* Qs = smem_raw + st * SM::STAGE;
-    const unsigned char* Bs = Qs + SM::Q_BYTES;
-    float acc[2][4][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int n = 0; n < 4; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
-
-    // one k16 step: A fragments (2 m-tiles) from tile `at` (rows of atb bytes, chunk ach),
-    // B fragments (4 n-tiles) from the SB tile at chunk bch
-    auto step = [&](const unsigned char* at, int atb, int ach, int bch, int nb) {
-      uint32_t a[2][4];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int r = wm * 32 + mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(at + swz(r, ach + (lane >> 4), atb)), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-      }
-      for (int u = 0; u < nb; ++u) {
-        const int bc = bch + 2 * u;
-#pragma unroll
-        for (int np = 0; np < 4; np += 2) {
-          uint32_t b0, b1, b2, b3;
-          const int r = wn * 32 + np * 8 + (lane & 7) + 8 * (lane >> 4);
-          ldsm_x4(smem_u32(Bs + swz(r, bc + ((lane >> 3) & 1), SB_ROWB)), b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16(acc[mt][np], a[mt], b0, b1);
-            mma_bf16(acc[mt][np + 1], a[mt], b2, b3);
-          }
-        }
-      }
-    };
-    // q . s_hi and q . s_lo: the q fragment is loaded once for both
-#pragma unroll 1
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t a[2][4];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int r = wm * 32 + mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(Qs + swz(r, 2 * ks + (lane >> 4), 256)), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-      }
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int bc = part * 16 + 2 * ks;
-#pragma unroll
-        for (int np = 0; np < 4; np += 2) {
-          uint32_t b0, b1, b2, b3;
-          const int r = wn * 32 + np * 8 + (lane & 7) + 8 * (lane >> 4);
-          ldsm_x4(smem_u32(Bs + swz(r, bc + ((lane >> 3) & 1), SB_ROWB)), b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16(acc[mt][np], a[mt], b0, b1);
-            mma_bf16(acc[mt][np + 1], a[mt], b2, b3);
-          }
-        }
-      }
-    }
-    // residual: t_hi . s'_hi + t_hi . s'_lo + t_lo . s'_hi
-#pragma unroll 1
-    for (int ks = 0; ks < R / 16; ++ks) {
-      step(TTs, TT_ROWB, 2 * ks, 32 + 2 * ks, 1);                 // t_hi . s'_hi
-      step(TTs, TT_ROWB, 2 * ks, 32 + R / 8 + 2 * ks, 1);         // t_hi . s'_lo
-      step(TTs, TT_ROWB, R / 8 + 2 * ks, 32 + 2 * ks, 1);         // t_lo . s'_hi
-    }
-    // epilogue for this head
-    const int h = g * G + hl;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int rloc = wm * 32 + mt * 16 + gq + 8 * hr, i = i0 + rloc;
-        const int p = Ps[rloc];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          const int cc = wn * 32 + n * 8 + 2 * tq, c = c0 + cc;
-          float z0 = (c < C && chunk_eligible(c, p, w)) ? tau * acc[mt][n][2 * hr] - lambda * Hs[hl][cc] : -INFINITY;
-          float z1 = (c + 1 < C && chunk_eligible(c + 1, p, w)) ? tau * acc[mt][n][2 * hr + 1] - lambda * Hs[hl][cc + 1]
-                                                                : -INFINITY;
-          zmax[mt][n][2 * hr] = fmaxf(zmax[mt][n][2 * hr], z0);
-          zmax[mt][n][2 * hr + 1] = fmaxf(zmax[mt][n][2 * hr + 1], z1);
-          if (i < Lq) {
-            float* zr = z_all + ((size_t)(b * Hq + h) * Lq + i) * C + c;
-            if (c + 1 < C) {
-              if (((C & 1) == 0)) *reinterpret_cast<float2*>(zr) = make_float2(z0, z1);
-              else { zr[0] = z0; zr[1] = z1; }
-            } else if (c < C) {
-              zr[0] = z0;
-            }
-          }
-        }
-      }
-    }
-    __syncthreads();   // stage `st` is refilled by the next iteration's prefetch
-  }
-  cp_async_wait<0>();
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int i = i0 + wm * 32 + mt * 16 + gq + 8 * hr;
-      if (i >= Lq) continue;
-      float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
-#pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        const int c = c0 + wn * 32 + n * 8 + 2 * tq;
-        if (c < C) zr[c] = zmax[mt][n][2 * hr];
-        if (c + 1 < C) zr[c + 1] = zmax[mt][n][2 * hr + 1];
-      }
-    }
   }
 }
 
