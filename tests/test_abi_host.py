@@ -124,3 +124,18 @@ def test_split_summary_layout_only_on_decode_blocks():
     it before launching anything."""
     dm = dims(flags=rdl.FLAG_SPLIT_SUMMARY)          # fp32, d = 64, prefill-shaped
     assert _score(dm) == rdl.ERR_UNSUPPORTED
+
+
+def test_decode_block_workspaces():
+    """A 32-query decode block over 128K: the attention keeps one fp32 output per chunk task
+    plus the window part per (row, head); the scorer the 8 hidden-slice partials of t and the
+    per-head scores.  The attention workspace fits the no-allocation scratch."""
+    dm = dims(L=131072, Lq=32, Hq=28, Hkv=4, d=128, D=3584, r=64, K=32, w=256)
+    rows = 32 * 28
+    want_attn = rows * 32 * 128 * 4 + rows * 128 * 4 + rows * 8
+    got_attn = rdl.workspace_bytes(rdl.WS_ATTN, dm, "bf16")
+    assert want_attn <= got_attn <= want_attn + 3 * 256            # three 256-byte aligned parts
+    assert got_attn < rdl.NOALLOC_SCRATCH_BYTES
+    want_score = 28 * 32 * 2048 * 4 + 8 * 32 * 64 * 4
+    got_score = rdl.workspace_bytes(rdl.WS_SCORE, dm, "bf16")
+    assert want_score <= got_score <= want_score + 2 * 256
