@@ -2,6 +2,7 @@
 // layout and kernel dispatch.  Nothing here allocates, frees or synchronises (apart from
 // rdl_last_device_status, which is documented to synchronise).
 #include <atomic>
+#include <mutex>
 #include <type_traits>
 #include <climits>
 #include <cstdint>
@@ -804,18 +805,54 @@ constexpr size_t kNoAllocScratchBytes = RDL_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+// (context id, address) per device: the address belongs to the module loaded into one
+// context, and context ids are unique for the life of the process, so a new primary context
+// on the device (after cudaDeviceReset) triggers a fresh lookup.
+struct NoAllocSlot {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
+NoAllocSlot g_noalloc_slot[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+// Id of the current context, 0 when none is current.
+unsigned long long current_context_id() {
+  typedef int (*CtxGetCurrentFn)(void**);                        // cuCtxGetCurrent
+  typedef int (*CtxGetIdFn)(void*, unsigned long long*);         // cuCtxGetId
+  static const CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device.  In host code the array's
 // name is only a host-side stand-in, so the address must come from cudaGetSymbolAddress,
-// looked up once per device with that device current (the first call on that device).
+// looked up with that device current: on the first call on that device, and again whenever
+// the device's context has changed since the last lookup.
 void* noalloc_scratch_ptr() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  unsigned long long id = current_context_id();     // 0 until the runtime has touched this device
+  if (id && slot.ptr && slot.ctx_id == id) return slot.ptr;
+  void* p = nullptr;
+  // also creates and binds the device's primary context when none is current yet
   if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-  g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  id = current_context_id();
+  if (!id) return nullptr;
+  slot.ctx_id = id;
+  slot.ptr = p;
   return p;
 }
 

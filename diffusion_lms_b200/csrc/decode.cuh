@@ -24,9 +24,12 @@
 //                     o = (e^lambda_loc o_loc + sum_c e^{z_c} o_c) / Z, in a fixed order.
 //
 // The kernels of one call are chained with programmatic dependent launch: every kernel
-// waits (griddepcontrol.wait) before it touches anything an earlier kernel writes, and
-// allows its dependent to launch only after that wait, so the early start of a dependent
-// never reads data older than the call's own inputs.
+// waits (griddepcontrol.wait) before it touches anything an earlier kernel writes (read
+// after write) and before its first store to a buffer an earlier kernel may still read
+// (write after read: two calls in a row on one workspace), and allows its dependent to
+// launch only after that wait, so the early start of a dependent never reads data older
+// than the call's own inputs nor overwrites data its predecessors still need.  Work that
+// reads only inputs of the call and writes only shared memory may run before the wait.
 #pragma once
 #include "common.cuh"
 #include "tc.cuh"
@@ -1176,9 +1179,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 // two rows x 8 head slots), and the warps' partial states are merged in a fixed order.
 // ROUTE_WIN: the local-window part of a route layer.  It reads only inputs of the call, so
 // it runs while the top-K of the same step is still running: it releases its dependent at
-// once and waits for its own predecessor only before it exits (its completion then implies
-// the predecessor's).  It writes the window's (max, sum) and unnormalised vector per
-// (row, head) for dec_comb_kernel instead of the normalised output.
+// once and waits for its own predecessor only before its first global store (its completion
+// then implies the predecessor's, and no store overtakes a read of the predecessor).  It
+// writes the window's (max, sum) and unnormalised vector per (row, head) for
+// dec_comb_kernel instead of the normalised output.
 // =====================================================================================
 constexpr int SW_WARPS = 6;
 
@@ -1354,6 +1358,10 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
   }
   // ---- fixed-order merge of the warps' states through shared memory (slabs are idle now)
   __syncthreads();
+  // ROUTE_WIN: the window part goes to a workspace the previous kernel on the stream may
+  // still be reading (the combine of an earlier call on the same workspace), so every store
+  // waits for the predecessor first; everything above touched inputs and shared memory only.
+  if (ROUTE_WIN) grid_dep_wait();
   float* part = reinterpret_cast<float*>(slabs) + warp * (16 * 128 + 64);   // [16 rows][128] + m, l
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) {
@@ -1405,7 +1413,6 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
     if (lse && d4 == 0) lse[(size_t)(b * Hq + h) * Lq + i] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
   }
   RDL_TRACE_POINT(5, 1);
-  if (ROUTE_WIN) grid_dep_wait();     // complete only after the predecessor (top-K) has
   (void)C;
 }
 

@@ -175,7 +175,8 @@ def rdl_route_attn(q, q_pos, k, v, idx, z_sel, dims: Dims, dtype, o, lse=None, w
 def rdl_route_attn_noalloc(q, q_pos, k, v, idx, z_sel, dims: Dims, dtype, o, lse=None,
                            stream=None, raise_on_error=True) -> int:
     """rdl_route_attn without a workspace argument: for hosts that cannot allocate device
-    memory at call time; librdl uses its own static device scratch (16 MiB per device)."""
+    memory at call time; librdl uses its own static device scratch of
+    NOALLOC_SCRATCH_BYTES per device."""
     s = _lib.rdl_route_attn_noalloc(_p(q), _p(q_pos), _p(k), _p(v), _p(idx), _p(z_sel),
                                     ctypes.byref(dims.c()), _dt(dtype), _p(o), _p(lse),
                                     _stream(stream))

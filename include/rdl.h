@@ -178,11 +178,15 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * and launches nothing (a 32-query decode block over 28 heads with K = 32 and a +-256 window
  * needs about 14.5 MiB).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- * with that device current); make that first call before any stream capture begins.
+ * with that device current); make that first call before any stream capture begins.  The
+ * address is kept per device and context: after cudaDeviceReset the next call on that
+ * device looks it up again (again before any capture).
  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
  * Every call on a device shares the one array and leaves its contents behind; no part of
- * it needs to start at zero.  Calls that overlap on the GPU (concurrent streams, or
- * several host threads) race on the array: serialise them.
+ * it needs to start at zero.  Calls issued one after another on one stream are safe (each
+ * call's kernels wait for the previous call's last reads of the array before writing it).
+ * Calls that overlap on the GPU (concurrent streams, or several host threads on different
+ * streams) race on the array: serialise them.
  */
 #define RDL_NOALLOC_SCRATCH_BYTES (32u << 20)
 rdl_status rdl_route_attn_noalloc(const void* q, const int32_t* q_pos, const void* k,
