@@ -5,7 +5,8 @@
 // the chunks), organised for the decode shape: the summaries s [Hq, C, d] (fp32, cached
 // across decode steps) dominate the bytes, so they are streamed from HBM exactly once.
 //
-//   decode_qres_kernel   q_res = q + (x W_down) W_up for each row (fp32), one CTA per row
+//   dec_tpart/dec_tsum/dec_qres   q_res = q + (x W_down) W_up for each row (fp32): the
+//                        weights are read once, slice by slice
 //   decode_score_kernel  per (64-chunk tile, KV group): for each head, the fp32 summaries
 //                        and residual queries are split into bf16 hi/lo terms in shared
 //                        memory and contracted on tensor cores,
@@ -15,81 +16,6 @@
 #include "common.cuh"
 
 namespace rdl {
-
-// --------------------------------------------------------------------------- q_res
-// One CTA (256 threads) per query row.  x row staged in shared memory; t = x W_down with
-// the D loop split across warps; q_res = q + t W_up with 256 threads over the Hq*d columns.
-template <typename T>
-__global__ void __launch_bounds__(256) decode_qres_kernel(const T* __restrict__ q, const T* __restrict__ x,
-                                                          const T* __restrict__ w_down,
-                                                          const T* __restrict__ w_up, int D, int r, int HD,
-                                                          float* __restrict__ qres) {
-  extern __shared__ float sm[];
-  float* xs = sm;                 // [D]
-  float* part = xs + D;           // [8][128]
-  float* ts = part + 8 * 128;     // [128]
-  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int k = tid; k < D; k += 256) xs[k] = x ? IO<T>::ld(x + (size_t)row * D + k) : 0.f;
-  __syncthreads();
-  if (r > 0 && x) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int k0 = (int)((long long)D * warp / 8), k1 = (int)((long long)D * (warp + 1) / 8);
-    // 8 rows of W_down per step: 8 independent loads per column in flight
-    int k = k0;
-    for (; k + 8 <= k1; k += 8) {
-      float wv[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          wv[j][u] = (lane + 32 * u < r) ? IO<T>::ld(w_down + (size_t)(k + j) * r + lane + 32 * u) : 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = fmaf(xs[k + j], wv[j][u], acc[u]);
-    }
-    for (; k < k1; ++k) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (lane + 32 * u < r) acc[u] = fmaf(xs[k], IO<T>::ld(w_down + (size_t)k * r + lane + 32 * u), acc[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (lane + 32 * u < r) part[warp * 128 + lane + 32 * u] = acc[u];
-    __syncthreads();
-    if (tid < r) {
-      float s = 0.f;
-      for (int w8 = 0; w8 < 8; ++w8) s += part[w8 * 128 + tid];
-      ts[tid] = s;
-    }
-    __syncthreads();
-  }
-  // columns in groups of 8 per thread: the 8 loads of one W_up row are independent
-  for (int c0 = tid; c0 < HD; c0 += 256 * 8) {
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = c0 + 256 * j;
-      v[j] = col < HD ? IO<T>::ld(q + (size_t)row * HD + col) : 0.f;
-    }
-    if (r > 0 && x) {
-      for (int m = 0; m < r; ++m) {
-        const float tm = ts[m];
-        const T* wr = w_up + (size_t)m * HD;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = c0 + 256 * j;
-          if (col < HD) v[j] = fmaf(tm, IO<T>::ld(wr + col), v[j]);
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = c0 + 256 * j;
-      if (col < HD) qres[(size_t)row * HD + col] = v[j];
-    }
-  }
-}
 
 // --------------------------------------------------------------------------- q_res, sliced
 // For few rows the weights dominate the bytes, so each CTA reads one slice of them once:

@@ -309,6 +309,52 @@ def check_shortage_and_group_max():
     assert np.all(np.isneginf(z[0, :, 0, 1:]))
 
 
+def check_scores_for():
+    """Per-head scores of a given selection (the parity check scores the GPU's own choice).
+
+    (a) Hand-worked, d = 2, one group of two heads, C = 3, query at position 10, no window,
+        rank-1 residual that adds (0, 1) to head 1 only:
+          head 0: q_res = (1, 0); head 1: q_res = (0, 2) + (0, 1) = (0, 3)
+          s[h0] = (1, 1), (2, 0), (0, 3);  H[h0] = 0.5, 1.0, 1.5
+          s[h1] = (0, 1), (1, 1), (-1, 0); H[h1] = 2.0, 0.0, 1.0
+        z = tau q_res.s - 0.1 H with tau = 1/sqrt(2); forced idx (2, 0, -1):
+          head 0: (-0.15, tau - 0.05, -inf);  head 1: (-0.1, 3 tau - 0.2, -inf).
+        With a window of radius 10 around position 10, chunk 0 touches the window: its
+        score is -inf for both heads whatever was forced.
+    (b) On the selection route_score_topk makes itself, the same scores it returned.
+    """
+    tau = 1.0 / math.sqrt(2.0)
+    q = np.zeros((1, 1, 2, 2))
+    q[0, 0, 0] = [1.0, 0.0]
+    q[0, 0, 1] = [0.0, 2.0]
+    x = np.ones((1, 1, 1))
+    wd = np.ones((1, 1))
+    wu = np.array([[0.0, 0.0, 0.0, 1.0]])
+    s = np.zeros((1, 2, 3, 2))
+    s[0, 0] = [[1, 1], [2, 0], [0, 3]]
+    s[0, 1] = [[0, 1], [1, 1], [-1, 0]]
+    H = np.array([[[0.5, 1.0, 1.5], [2.0, 0.0, 1.0]]])
+    idx = np.array([[[[2, 0, -1]]]])
+    z = O.scores_for(q, np.array([[10]]), x, wd, wu, s, H, idx, w=-1, lam=0.1, L=192)
+    exp = np.array([[-0.15, tau - 0.05, -np.inf], [-0.1, 3 * tau - 0.2, -np.inf]])
+    assert np.allclose(z[0, :, 0], exp, atol=1e-14), z[0, :, 0]
+    assert np.array_equal(np.isneginf(z[0, :, 0]), np.isneginf(exp))
+    zw = O.scores_for(q, np.array([[10]]), x, wd, wu, s, H, idx, w=10, lam=0.1, L=192)
+    assert np.isneginf(zw[0, :, 0, 1]).all()
+    assert np.allclose(zw[0, :, 0, 0], exp[:, 0], atol=1e-14)
+    # (b) agreement with the scores the selection step attaches to its own choice
+    cs = _route_case(13, L=448, w=30, K=3)
+    q, k, v = cs["q"], cs["k"], cs["v"]
+    s, H, _ = O.summary_pool(q[:, O.S - 1::O.S], k, v)
+    rows = np.arange(0, cs["L"], 5)
+    idx, z_sel = O.route_score_topk(q, None, cs["x"], cs["wd"], cs["wu"], s, H, Hkv=cs["Hkv"],
+                                    K=cs["K"], w=cs["w"], lam=cs["lam"], rows=rows)
+    z2 = O.scores_for(q, None, cs["x"], cs["wd"], cs["wu"], s, H, idx, w=cs["w"], lam=cs["lam"],
+                      rows=rows)
+    content = [i for i in rows if not O.is_mask_slot(i)]
+    assert np.array_equal(z2[:, :, content], z_sel[:, :, content])
+
+
 # ----------------------------------------------------------------------------- attention
 
 def _sdpa(qv, keys, vals, bias=None):
@@ -511,6 +557,7 @@ ALL_CHECKS = [
     check_pool_closed_forms, check_pool_shift_invariance, check_pool_gqa_and_mean,
     check_pool_peaked_cosine, check_residual_layout, check_score_hand_example,
     check_topk_bruteforce, check_selection_properties, check_shortage_and_group_max,
+    check_scores_for,
     check_partition_identity, check_masses_sum_to_one, check_special_cases, check_swa_band,
     check_locality, check_two_chunk_hand_examples,
 ]

@@ -85,7 +85,29 @@ def _row_unnormalised_chunk(q_i, p, k_g, v_g, chunks, z_c, w):
     return o * 1.01, lnZ
 
 
+_real_scores_for = O.scores_for
+
+
+def _scores_for_heads_reversed(q, q_pos, x, w_down, w_up, s, H, idx, **kw):
+    """Mistake: the heads of each group are read in reverse order."""
+    z = _real_scores_for(q, q_pos, x, w_down, w_up, s, H, idx, **kw)
+    Hkv = idx.shape[1]
+    G = z.shape[1] // Hkv
+    return z.reshape(z.shape[0], Hkv, G, *z.shape[2:])[:, :, ::-1].reshape(z.shape)
+
+
+def _scores_for_group_max(q, q_pos, x, w_down, w_up, s, H, idx, **kw):
+    """Mistake: every head of a group gets the group-max score."""
+    z = _real_scores_for(q, q_pos, x, w_down, w_up, s, H, idx, **kw)
+    Hkv = idx.shape[1]
+    G = z.shape[1] // Hkv
+    zg = z.reshape(z.shape[0], Hkv, G, *z.shape[2:]).max(axis=2, keepdims=True)
+    return np.broadcast_to(zg, (z.shape[0], Hkv, G) + z.shape[2:]).reshape(z.shape)
+
+
 MUTATIONS = {
+    "scores_for_heads_reversed": ("scores_for", _scores_for_heads_reversed),
+    "scores_for_group_max": ("scores_for", _scores_for_group_max),
     "tau_1_over_d": ("tau_of", _tau_wrong),
     "window_exclusive": ("window", _window_exclusive),
     "eligible_ignores_window": ("eligible", _eligible_own_chunk_only),

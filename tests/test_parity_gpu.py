@@ -83,6 +83,58 @@ def test_bf16_many_scattered_rows_partial_tiles():
     P.check_swa(wl, gpu, rows)
 
 
+def test_bf16_prefill_batch_2_every_row():
+    """Two independently drawn sequences (B = 2) through the tensor-core prefill kernels at
+    head dim 128 (scorer, window and chunk attention index across the batch), every row."""
+    wl = W.make_inputs(small(B=2), seed=31, n_needles=4)
+    assert not np.array_equal(wl.k[0], wl.k[1]) and not np.array_equal(wl.q[0], wl.q[1])
+    assert not np.array_equal(wl.needles[0], wl.needles[1])
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(wl.dims.L)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_exact"] > 2000
+    P.check_swa(wl, gpu, rows)
+    assert not np.array_equal(gpu["idx"][0], gpu["idx"][1])
+
+
+@pytest.mark.parametrize("dtype,r,D", [("f32", 64, 512), ("bf16", 16, 512), ("bf16", 64, 520)])
+def test_decode_block_general_scorer(dtype, r, D):
+    """Decode blocks outside the chained tensor-core scorer's shapes (fp32 storage, a rank
+    other than 0/64/128, a hidden size not a multiple of 64) take the general decode
+    scorer: sliced residual, split-bf16 summary contraction, group max, top-K."""
+    dm = small(L=8192, Lq=32, K=16, w=256, r=r, D=D, dtype=dtype)
+    wl = W.make_inputs(dm, seed=32, n_needles=6, decode_block=32, unit_scale=(dtype == "f32"))
+    gpu = P.run_gpu(wl, swa=True)
+    rows = np.arange(32)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+def test_window_radius_1280_prefill_sampled():
+    """The window radius of the pages' Table 3 layout for the non-route layers (1280), on a
+    prefill: route layer and sliding window, sampled rows including both ends."""
+    dm = small(L=4096, Lq=4096, K=8, w=1280)
+    wl = W.make_inputs(dm, seed=33, n_needles=4)
+    gpu = P.run_gpu(wl, swa=True)
+    rows = P.sample_rows(wl, 400, seed=3)
+    P.check_route_layer(wl, gpu, rows)
+    P.check_swa(wl, gpu, rows)
+
+
+def test_window_radius_1280_decode_stack_layers():
+    """A route layer and a sliding-window layer of the 128K stack with radius 1280."""
+    for layer in (2, 3):
+        wl = W.stack_layer(layer)
+        wl = dataclasses.replace(wl, dims=dataclasses.replace(wl.dims, w=1280))
+        route = W.is_route_layer(layer)
+        gpu = P.run_gpu(wl, route=route, swa=not route)
+        rows = np.arange(32)
+        if route:
+            P.check_route_layer(wl, gpu, rows)
+        else:
+            P.check_swa(wl, gpu, rows)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(16, 2), (2, 2), (6, 1)])
 def test_group_sizes(Hq, Hkv):
     wl = W.make_inputs(small(L=1024, Lq=1024, Hq=Hq, Hkv=Hkv, K=6, w=70), seed=14, n_needles=2)
@@ -102,7 +154,8 @@ def test_bf16_head_dim_64_batch_2():
 
 
 @pytest.mark.parametrize("case", ["no_window", "window_covers_all", "lambda0_no_residual",
-                                  "mean_summary", "K_equals_C"])
+                                  "lambda0_with_residual", "no_residual", "mean_summary",
+                                  "K_equals_C"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_edge_cases(case, dtype):
     kw = dict(L=1024, Lq=1024, Hq=8, Hkv=2, K=4, w=64, dtype=dtype)
@@ -113,6 +166,10 @@ def test_edge_cases(case, dtype):
         kw["w"] = 5000
     elif case == "lambda0_no_residual":
         kw["lam"] = 0.0
+        with_res = False
+    elif case == "lambda0_with_residual":        # Table 6 "No entropy"
+        kw["lam"] = 0.0
+    elif case == "no_residual":                  # Table 6 "No residual"
         with_res = False
     elif case == "mean_summary":
         flags, mean = rdl.FLAG_MEAN_SUMMARY, True
