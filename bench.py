@@ -30,15 +30,37 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "route-layer sparse-attn query-tokens/s at 16K-128K; decode-step ms at 128K"
-# DRAM bytes of one rdl_route_attn call on the 16K prefill (window + chunk kernels), from one
-# ncu capture of the current kernels; set to None when either kernel changes.
-ATTN_PREFILL_TRAFFIC = 941.8e6
-# DRAM bytes of one 128K decode step (the six decode kernels, one launch each, caches cold
-# between kernels under ncu, so intermediates re-read from DRAM here stay in L2 live); set to
-# None when a decode kernel changes.
-DECODE_STEP_TRAFFIC = 108.34e6
+# DRAM traffic of the dominant kernels from ncu captures, each entry keyed by the hash of the
+# library sources it was taken on; an entry whose hash differs from the current sources is
+# stale and reported as null.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 UNIT = "query-tokens/s"
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def kernel_sources_sha() -> str:
+    """sha256 (16 hex digits) of the CUDA library sources and the C header."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "diffusion_lms_b200", "csrc", "*.cu*")))
+    for f in files + [os.path.join(ROOT, "include", "rdl.h")]:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(key: str):
+    """(bytes per launch or None, note) for `key`, if captured on the current sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no ncu capture recorded"
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f).get(key)
+    if rec is None:
+        return None, "no ncu capture recorded for this kernel"
+    if rec.get("sources_sha") != kernel_sources_sha():
+        return None, "kernel sources changed since the last ncu capture"
+    return float(rec["bytes"]), rec.get("what", "")
 
 
 def peaks():
@@ -167,48 +189,120 @@ def job_throughput(rows_per_rank: int, world: int, ms_max: float) -> float:
 
 
 # ----------------------------------------------------------------------------- oracle arm
+#
+# The fp64 oracle as it stands, run on the host's cores: spawn-started worker processes (one
+# BLAS thread each) pool the summaries of a share of the heads, then score, select and attend
+# a share of the sampled rows.  Each worker receives the stored (bf16 bit) inputs it needs and
+# calls only oracle functions; the parent measures the wall time of both phases.
 
-def oracle_sample(wl, n_rows: int, seed: int = 0):
-    """Time the fp64 oracle on a bounded sample of the workload: all summaries + n rows."""
+MAX_ORACLE_WORKERS = 64
+_ORACLE_WL = {}
+
+
+def oracle_workers() -> int:
+    return max(1, min(os.cpu_count() or 1, MAX_ORACLE_WORKERS))
+
+
+def _oracle_init(arrays):
+    """Worker start-up: keep the workload's stored inputs (sent once per worker)."""
+    _ORACLE_WL.clear()
+    _ORACLE_WL.update(arrays)
+
+
+def _oracle_pool_heads(task):
     from threadpoolctl import threadpool_limits
     from oracle import rdl_oracle as O
     from diffusion_lms_b200.workloads import as_f64
-    f = {n: as_f64(getattr(wl, n)) for n in ("q", "q_mask", "k", "v", "x", "w_down", "w_up")}
-    dm = wl.dims
-    rng = np.random.default_rng(seed)
-    pos = np.arange(dm.L) if wl.q_pos is None else wl.q_pos[0]
-    cand = np.array([i for i in range(dm.Lq) if pos[i] % 64 != 63])
-    rows = np.sort(rng.choice(cand, size=min(n_rows, cand.size), replace=False))
+    heads, G = task
     with threadpool_limits(limits=1):
+        qm = as_f64(_ORACLE_WL["q_mask"][:, :, heads])
+        out = []
+        for j, h in enumerate(heads):
+            kf = as_f64(_ORACLE_WL["k"][:, h // G:h // G + 1])
+            s, H, _ = O.summary_pool(qm[:, :, j:j + 1], kf)
+            out.append((h, s[:, 0], H[:, 0]))
+    return out
+
+
+def _oracle_rows(task):
+    from threadpoolctl import threadpool_limits
+    from oracle import rdl_oracle as O
+    from diffusion_lms_b200.workloads import as_f64
+    rows, pos, s, H, kw = task
+    wl = _ORACLE_WL
+    with threadpool_limits(limits=1):
+        qf = as_f64(wl["q"][:, rows])
+        idx, z = O.route_score_topk(qf, pos, as_f64(wl["x"][:, rows]), as_f64(wl["w_down"]),
+                                    as_f64(wl["w_up"]), s, H, Hkv=kw["Hkv"], K=kw["K"],
+                                    w=kw["w"], lam=kw["lam"], L=kw["L"])
+        O.route_attn(qf, pos, as_f64(wl["k"]), as_f64(wl["v"]), idx, z, w=kw["w"])
+    return int(rows.size)
+
+
+class OracleRunner:
+    """Spawn-started worker pool timing the oracle on bounded samples of one workload."""
+
+    def __init__(self, wl, workers: int):
+        import multiprocessing as mp
+        self.wl = wl
+        self.workers = workers
+        arrays = {n: getattr(wl, n) for n in ("q", "q_mask", "k", "v", "x", "w_down", "w_up")}
+        self.pool = mp.get_context("spawn").Pool(workers, initializer=_oracle_init,
+                                                 initargs=(arrays,))
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+    def sample(self, n_rows: int, seed: int = 0):
+        """(seconds, rows): all summaries of the sequence + n random content rows."""
+        wl = self.wl
+        dm = wl.dims
+        G = dm.Hq // dm.Hkv
+        rng = np.random.default_rng(seed)
+        pos_all = np.arange(dm.L) if wl.q_pos is None else wl.q_pos[0]
+        cand = np.flatnonzero(pos_all[:dm.Lq] % 64 != 63)
+        rows = np.sort(rng.choice(cand, size=min(n_rows, cand.size), replace=False))
+        nw = self.workers
+        kw = dict(Hkv=dm.Hkv, K=dm.K, w=dm.w, lam=dm.lam, L=dm.L)
         t0 = time.perf_counter()
-        s, H, _ = O.summary_pool(f["q_mask"], f["k"], f["v"])
-        idx, z = O.route_score_topk(f["q"], wl.q_pos, f["x"], f["w_down"], f["w_up"], s, H,
-                                    Hkv=dm.Hkv, K=dm.K, w=dm.w, lam=dm.lam, L=dm.L, rows=rows)
-        O.route_attn(f["q"], wl.q_pos, f["k"], f["v"], idx, z, w=dm.w, rows=rows)
-        dt = time.perf_counter() - t0
-    return dt, rows.size
+        head_sets = [list(range(dm.Hq))[i::nw] for i in range(nw)]
+        s = np.zeros((dm.B, dm.Hq, dm.C, dm.d))
+        H = np.zeros((dm.B, dm.Hq, dm.C))
+        for part in self.pool.map(_oracle_pool_heads, [(hs, G) for hs in head_sets if hs]):
+            for h, sh, Hh in part:
+                s[:, h], H[:, h] = sh, Hh
+        tasks = [(r, pos_all[r][None, :].astype(np.int64), s, H, kw)
+                 for r in np.array_split(rows, nw) if r.size]
+        done = sum(self.pool.map(_oracle_rows, tasks))
+        return time.perf_counter() - t0, done
 
 
 def run_reference(args, rank):
+    """The oracle arm: the fp64 oracle on the host's cores, each step a bounded sample of the
+    16K prefill route layer (all summaries + ref_rows content rows)."""
     from diffusion_lms_b200 import workloads as W
     if rank != 0:
         return
     wl = W.prefill_16k()
-    n = args.ref_rows
+    runner = OracleRunner(wl, oracle_workers())
+    n = args.ref_rows if args.ref_rows > 0 else 16 * runner.workers
     for _ in range(args.warmup):
-        oracle_sample(wl, max(1, n // 8))
-    times = [oracle_sample(wl, n, seed=s)[0] for s in range(args.steps)]
-    ms = 1e3 * statistics.mean(times)
+        runner.sample(max(runner.workers, n // 8))
+    times = [runner.sample(n, seed=s_)[0] for s_ in range(args.steps)]
+    runner.close()
+    ms = 1e3 * statistics.median(times)
     val = n / (ms / 1e3)
     sample = (f"all 256x28 summaries + {n} random content rows of the 16K prefill per step "
-              f"(fp64 NumPy, 1 BLAS thread)")
+              f"(fp64 NumPy oracle, {runner.workers} spawn-started processes x 1 BLAS thread; "
+              f"host has {os.cpu_count()} cores)")
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": wl.name, "L": 16384, "Hq": 28, "Hkv": 4, "d": 128, "K": 32,
                        "w": 256, "r": 64, "D": 3584, "rows_per_step": n},
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": runner.workers, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -268,6 +362,7 @@ def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
     d_ms = max_over_ranks(float(np.median(gms)), world, dev) if world > 1 else float(np.median(gms))
     assert rdl.rdl_last_device_status() == rdl.OK
     db = decode_bytes(dinp.dims, dout.idx.cpu().numpy())
+    d_traffic, d_traffic_note = recorded_traffic("route_decode_128k.step")
     d_ach = db["total"] / (d_ms / 1e3) / 1e9
     del g
     return {"workload": wd.name, "ms_per_step": d_ms, "timing": "CUDA-graph replay, median",
@@ -276,10 +371,7 @@ def decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind):
             "query_tokens_per_s": world * 32 / (d_ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": d_ach / pk["hbm_gbs"], "algorithmic_bytes": db["total"],
-                         "traffic": DECODE_STEP_TRAFFIC,
-                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the six "
-                                           "decode kernels, one launch each "
-                                           "(profiles/launches_route_decode_128k.md)",
+                         "traffic": d_traffic, "traffic_source": d_traffic_note,
                          "unique_group_chunk_pairs": db["unique_pairs"],
                          "peak_source": f"hbm_gbs ({pk_kind})"}}
 
@@ -413,6 +505,99 @@ def stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind):
                          "peak_source": f"hbm_gbs ({pk_kind})"}}
 
 
+# ----------------------------------------------------------------------------- prefill
+
+def time_prefill(api, inp, out, stream, flush, steps, warmup, events=True):
+    """Per-step CUDA-event times [steps, 3] (summary pool, score + top-K, attention) of a
+    route-layer prefill step, L2 flushed before every step (untimed)."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        api.route_layer(inp, out, stream=stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for s_ in range(steps):
+        flush.zero_()
+        e = ev[s_]
+        e[0].record(stream)
+        api.summary_pool(inp, out, stream=stream)
+        e[1].record(stream)
+        api.score_topk(inp, out, stream=stream)
+        e[2].record(stream)
+        api.route_attn(inp, out, stream=stream)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    return np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev])
+
+
+def prefill_roofline(dims, idx, call_ms, step_ms, pk, pk_kind, traffic_key):
+    """Roofline of the dominant call (the attention call, window + chunk launches) and of the
+    whole step, both against the measured bf16 burst peak."""
+    fl_attn = attn_flops(dims, None, idx)
+    fl_score = score_flops(dims)
+    ach = fl_attn / (call_ms[2] / 1e3) / 1e12
+    traffic, note = recorded_traffic(traffic_key)
+    roof = {"kernel": "rdl_route_attn (window + chunk launches)", "bound": "tensor",
+            "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": ach / pk["bf16_tflops"], "traffic": traffic,
+            "traffic_source": note, "algorithmic_flops": fl_attn,
+            "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
+    step_fl = fl_attn + fl_score
+    step_ach = step_fl / (step_ms / 1e3) / 1e12
+    step = {"bound": "tensor", "algorithmic_flops": step_fl, "achieved": step_ach,
+            "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": step_ach / pk["bf16_tflops"]}
+    return roof, step
+
+
+def prefill_variants(args, api, rdl, wl, dev, stream, flush, world, max_ranks):
+    """The 16K prefill step with the ablations of the pages' Table 6 (mean summary, no
+    entropy, no residual) beside the default, each timed like the headline step."""
+    import torch
+    res = {}
+    for name, mod in (("mean_summary", dict(flags=rdl.FLAG_MEAN_SUMMARY)),
+                      ("no_entropy", dict(lam=0.0)), ("no_residual", dict(r=0))):
+        inp = api.to_device(wl, dev)
+        for k_, v_ in mod.items():
+            setattr(inp.dims, k_, v_)
+        if mod.get("r") == 0:
+            inp.x = None
+        out = api.alloc_outputs(inp.dims, inp.dtype, dev)
+        per = time_prefill(api, inp, out, stream, flush, max(3, args.steps // 2), args.warmup)
+        ms = max_ranks(float(np.median(per.sum(axis=1))))
+        assert rdl.rdl_last_device_status() == rdl.OK
+        res[name] = {"ms_per_step": ms, "query_tokens_per_s": world * 16128 / (ms / 1e3),
+                     "breakdown_ms": {"rdl_summary_pool": float(np.median(per[:, 0])),
+                                      "rdl_route_score_topk": float(np.median(per[:, 1])),
+                                      "rdl_route_attn": float(np.median(per[:, 2]))}}
+        del inp, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def prefill_long_bench(make_wl, args, api, rdl, dev, stream, flush, world, max_ranks, pk, pk_kind):
+    """A longer route-layer prefill (64K mixture keys, 128K), timed like the 16K step."""
+    import torch
+    wl = make_wl()
+    inp = api.to_device(wl, dev)
+    out = api.alloc_outputs(inp.dims, inp.dtype, dev)
+    per = time_prefill(api, inp, out, stream, flush, max(3, args.steps // 2), args.warmup)
+    ms = max_ranks(float(np.median(per.sum(axis=1))))
+    assert rdl.rdl_last_device_status() == rdl.OK
+    call_ms = np.median(per, axis=0)
+    rows = int(((np.arange(wl.dims.L) % 64) != 63).sum())
+    roof, step = prefill_roofline(wl.dims, out.idx.cpu().numpy(), call_ms, ms, pk, pk_kind,
+                                  f"{wl.name}.rdl_route_attn")
+    res = {"workload": wl.name, "ms_per_step": ms, "query_tokens_per_s": world * rows / (ms / 1e3),
+           "content_rows": rows, "timing": "median of per-step CUDA events, L2 flushed between",
+           "breakdown_ms": {"rdl_summary_pool": float(call_ms[0]),
+                            "rdl_route_score_topk": float(call_ms[1]),
+                            "rdl_route_attn": float(call_ms[2])},
+           "roofline": roof, "step_roofline": step}
+    del inp, out
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def main():
@@ -421,10 +606,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=96)
-    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="oracle rows per reference step (0: 16 per worker process)")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="oracle rows of the CPU baseline (0: 48 per worker process)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--no-64k", action="store_true")
+    ap.add_argument("--no-128k", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--stack-only", action="store_true",
                     help="time only the 28-layer 128K stack (profiling aid)")
     ap.add_argument("--decode-only", action="store_true",
@@ -441,6 +631,13 @@ def main():
         run_reference(args, rank)
         return
 
+    # the oracle's worker processes start (spawn) before any GPU work of this process
+    from diffusion_lms_b200 import workloads as W
+    wl = W.prefill_16k(seed=rank_seed(2, rank))
+    runner = None
+    if rank == 0 and not args.no_cpu_baseline:
+        runner = OracleRunner(wl, oracle_workers())
+
     import torch
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
@@ -451,7 +648,6 @@ def main():
                                 device_id=dev)
 
     from diffusion_lms_b200 import api, rdl
-    from diffusion_lms_b200 import workloads as W
 
     def barrier():
         if world > 1:
@@ -476,75 +672,32 @@ def main():
         return
 
     # ---------------- 16K prefill route layer (the headline workload)
-    wl = W.prefill_16k(seed=rank_seed(2, rank))
     inp = api.to_device(wl, dev)
     out = api.alloc_outputs(inp.dims, inp.dtype, dev)
-
-    def step():
-        api.route_layer(inp, out, stream=stream)
-
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        api.route_layer(inp, out, stream=stream)
     torch.cuda.synchronize()
     assert rdl.rdl_last_device_status() == rdl.OK
 
-    n_evt = 4
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_evt)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     barrier()
     torch.cuda.synchronize()
     launches0 = rdl.launch_count()
-    for s_ in range(args.steps):
-        flush.zero_()                       # L2 flushed between timed steps (not timed)
-        e = ev[s_]
-        e[0].record(stream)
-        api.summary_pool(inp, out, stream=stream)
-        e[1].record(stream)
-        api.score_topk(inp, out, stream=stream)
-        e[2].record(stream)
-        api.route_attn(inp, out, stream=stream)
-        e[3].record(stream)
-    torch.cuda.synchronize()
+    per = time_prefill(api, inp, out, stream, flush, args.steps, 0)
     launches = rdl.launch_count() - launches0
     barrier()
     clk = clocks.stop()
-    per = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_evt - 1)] for e in ev])
-    ms_step_local = float(per.sum(axis=1).mean())
-    ms_step = max_ranks(ms_step_local)
+    ms_step = max_ranks(float(np.median(per.sum(axis=1))))
     content_rows = int(((np.arange(wl.dims.L) % 64) != 63).sum())
     value = job_throughput(content_rows, world, ms_step)
-    call_ms = per.mean(axis=0)
+    call_ms = np.median(per, axis=0)
     assert rdl.rdl_last_device_status() == rdl.OK
-
-    idx_np = out.idx.cpu().numpy()
-    fl_attn = attn_flops(wl.dims, None, idx_np)
-    fl_score = score_flops(wl.dims)
     calls = {"rdl_summary_pool": float(call_ms[0]), "rdl_route_score_topk": float(call_ms[1]),
              "rdl_route_attn": float(call_ms[2])}
-    dominant = max(calls, key=calls.get)
-    if dominant == "rdl_route_attn":
-        achieved = fl_attn / (call_ms[2] / 1e3) / 1e12
-        roof = {"kernel": "rdl_route_attn (window + chunk launches)", "bound": "tensor",
-                "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops"], "traffic": ATTN_PREFILL_TRAFFIC,
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                  "window_tc_kernel<1> + chunk_tc_kernel, one launch each "
-                                  "(profiles/attn_traffic_route_prefill_16k.md)",
-                "algorithmic_flops": fl_attn, "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
-    elif dominant == "rdl_route_score_topk":
-        achieved = fl_score / (call_ms[1] / 1e3) / 1e12
-        roof = {"kernel": "rdl_route_score_topk", "bound": "tensor", "achieved": achieved,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                "traffic": None, "algorithmic_flops": fl_score,
-                "peak_source": f"bf16_tflops ({pk_kind}, burst)"}
-    else:
-        by = 2 * 2 * wl.dims.Hkv * wl.dims.L * wl.dims.d + 4 * wl.dims.Hq * (wl.dims.L // 64) * (wl.dims.d + 1)
-        achieved = by / (call_ms[0] / 1e3) / 1e9
-        roof = {"kernel": "rdl_summary_pool", "bound": "hbm", "achieved": achieved,
-                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                "traffic": None, "peak_source": f"hbm_gbs ({pk_kind})"}
+    roof, step_roof = prefill_roofline(wl.dims, out.idx.cpu().numpy(), call_ms, ms_step, pk,
+                                       pk_kind, "route_prefill_16k.rdl_route_attn")
 
     # ---------------- end to end through the public API with host buffers
     pin = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "x", "w_down", "w_up")}
@@ -574,26 +727,38 @@ def main():
     e2e_ms = max_ranks(e0.elapsed_time(e1) / n_e2e)
     e2e = {"value": job_throughput(content_rows, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-    del pin, h_o, h_idx
+    del pin, h_o, h_idx, inp, out
+    torch.cuda.empty_cache()
 
+    variants = None
+    if not args.no_variants:
+        variants = prefill_variants(args, api, rdl, wl, dev, stream, flush, world, max_ranks)
+    p64 = p128 = None
+    if not args.no_64k:
+        p64 = prefill_long_bench(lambda: W.prefill_64k(seed=rank_seed(4, rank)), args, api, rdl,
+                                 dev, stream, flush, world, max_ranks, pk, pk_kind)
+    if not args.no_128k:
+        p128 = prefill_long_bench(lambda: W.prefill_128k(seed=rank_seed(6, rank)), args, api, rdl,
+                                  dev, stream, flush, world, max_ranks, pk, pk_kind)
     # ---------------- 128K decode block (summaries cached; score + attention)
     decode = None
     if not args.no_decode:
-        del inp, out
-        torch.cuda.empty_cache()
         decode = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
     stack = None
     if not args.no_stack:
         torch.cuda.empty_cache()
         stack = stack_bench(args, dev, stream, flush, rank, world, pk, pk_kind)
 
-    # ---------------- CPU baseline (rank 0, oracle on a bounded sample)
+    # ---------------- CPU baseline (rank 0, the oracle on a bounded sample, all worker cores)
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
-        dt, n = oracle_sample(wl, args.cpu_rows)
-        cpu = {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+    if runner is not None:
+        n = args.cpu_rows if args.cpu_rows > 0 else 48 * runner.workers
+        dt, n = runner.sample(n)
+        runner.close()
+        cpu = {"value": n / dt, "unit": UNIT, "cores": runner.workers, "kind": "oracle",
                "sample": f"all 256x28 summaries + {n} random content rows of the 16K prefill "
-                         f"(fp64 NumPy, 1 BLAS thread), {dt:.1f} s"}
+                         f"(fp64 NumPy oracle, {runner.workers} spawn-started processes x 1 BLAS "
+                         f"thread; host has {os.cpu_count()} cores), {dt:.1f} s"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -603,9 +768,12 @@ def main():
                 "config": {"workload": wl.name, "L": 16384, "Hq": 28, "Hkv": 4, "d": 128, "K": 32,
                            "w": 256, "r": 64, "D": 3584, "content_rows": content_rows,
                            "l2": "flushed between timed steps (256 MB write, untimed)",
+                           "timing": "median of per-step CUDA events",
                            "parallelism": f"independent sequence per GPU x{world}"},
-                "breakdown_ms": calls, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk, "decode_128k": decode, "stack_128k": stack}
+                "breakdown_ms": calls, "roofline": roof, "step_roofline": step_roof,
+                "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk, "prefill_64k": p64, "prefill_128k": p128,
+                "prefill_16k_variants": variants, "decode_128k": decode, "stack_128k": stack}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

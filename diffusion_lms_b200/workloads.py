@@ -213,6 +213,8 @@ DECODE_128K = Dims(B=1, L=131072, Lq=32, Hq=28, Hkv=4, d=128, D=3584, r=64, K=32
                    w=256, lam=0.1, dtype="bf16")
 PREFILL_64K = Dims(B=1, L=65536, Lq=65536, Hq=28, Hkv=4, d=128, D=3584, r=64, K=32,
                    w=256, lam=0.1, dtype="bf16")
+PREFILL_128K = Dims(B=1, L=131072, Lq=131072, Hq=28, Hkv=4, d=128, D=3584, r=64, K=32,
+                    w=256, lam=0.1, dtype="bf16")
 STACK_LAYERS = 28
 STACK_ROUTE_EVERY = 4          # route layer when layer % 4 == 3
 
@@ -236,6 +238,11 @@ def decode_128k(seed: int = 3) -> Workload:
 def prefill_64k(seed: int = 4) -> Workload:
     """Route layer prefill at 64K with keys from a 32-component mixture (near-tie top-K)."""
     return make_inputs(PREFILL_64K, seed=seed, mixture=32, name="route_prefill_64k_mixture")
+
+
+def prefill_128k(seed: int = 6) -> Workload:
+    """Route-layer prefill at 128K (the top of the 16K-128K range), bf16, 16 needles."""
+    return make_inputs(PREFILL_128K, seed=seed, n_needles=16, name="route_prefill_128k")
 
 
 def stack_layer(layer: int, seed: int = 5) -> Workload:

@@ -294,6 +294,21 @@ def test_prefill_64k_mixture_sampled():
     assert r["n_tie"] > 0          # the mixture keys create near ties
 
 
+def test_prefill_128k_sampled():
+    """Route-layer prefill at 128K: summaries of all 2048 chunks, 512 sampled rows (first
+    and last chunks, window edges, rows next to needles), properties on every row."""
+    wl = W.prefill_128k()
+    gpu = P.run_gpu(wl)
+    rows = P.sample_rows(wl, 512, seed=2)
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_exact"] > 1000
+    idx = gpu["idx"][0]
+    assert idx.shape == (4, 131072, 32) and idx.max() < 2048
+    content = (np.arange(131072) % 64) != 63
+    assert np.all(idx[:, ~content] == -1) and np.all(idx[:, content] >= 0)
+    assert np.all(np.isfinite(gpu["o"])) and np.all(np.isfinite(gpu["lse"][:, :, content]))
+
+
 def test_stack_128k_all_layers():
     for layer in range(W.STACK_LAYERS):
         wl = W.stack_layer(layer)
