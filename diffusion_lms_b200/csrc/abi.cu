@@ -17,6 +17,7 @@
 #include "chunk_attn.cuh"
 #include "tmap.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_major.cuh"
 #include "window_tc.cuh"
 #include "score_tc.cuh"
 #include "decode.cuh"
@@ -88,6 +89,11 @@ constexpr int kFastScoreMinRows = 128;
 bool fast_score(const rdl_dims* dm, rdl_dtype t) {
   return t == RDL_BF16 && dm->d == 128 && dm->r == 64 && dm->D % 64 == 0 && dm->Hq / dm->Hkv <= 8 &&
          dm->Lq >= kFastScoreMinRows;
+}
+// The tensor-core scorer in two passes around the top-K, without a per-head score buffer, once
+// that buffer would pass 1 GiB (long sequences); below, one pass writing every per-head score.
+bool fused_score(const rdl_dims* dm, rdl_dtype t) {
+  return fast_score(dm, t) && sizeof(float) * (size_t)dm->B * dm->Hq * dm->Lq * (dm->L / S) > (size_t(1) << 30);
 }
 // decode blocks: few rows, head dim 128 -> the decode score path
 bool decode_score_path(const rdl_dims* dm) { return dm->d == 128 && dm->Lq <= 64; }
@@ -180,12 +186,23 @@ ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
   const size_t C = dm->L / S;
   ScoreWs w{};
   size_t off = 0;
+  if (fused_score(dm, dt)) {
+    // the group maxima, the split residual rows and the split summary rows (no per-head scores)
+    w.zeta = off; off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
+    w.tt = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Lq * 2 * dm->r);
+    w.sb = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Hq * C * (2 * dm->d + 2 * dm->r));
+    w.total = off;
+    return w;
+  }
   w.z_all = off; off += align256(sizeof(float) * (size_t)dm->B * dm->Hq * dm->Lq * C);
   w.zeta = off;
-  if (!dec_score_ok(dm, dt)) off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
   if (dec_score_ok(dm, dt)) {
     // the hidden-slice partials of t, summed by the scorer
     w.t = off;     off += align256(sizeof(float) * dec::TK_CL * (size_t)dm->B * dm->Lq * (dm->r > 0 ? dm->r : 1));
+  } else {
+    off += align256(sizeof(float) * (size_t)dm->B * dm->Hkv * dm->Lq * C);
+  }
+  if (dec_score_ok(dm, dt)) {
   } else if (fast_score(dm, dt)) {
     w.tt = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Lq * 2 * dm->r);
     w.sb = off;  off += align256(sizeof(__nv_bfloat16) * (size_t)dm->B * dm->Hq * C * (2 * dm->d + 2 * dm->r));
@@ -202,7 +219,23 @@ ScoreWs score_ws(const rdl_dims* dm, rdl_dtype dt) {
 }
 struct AttnWs {
   size_t o_loc, lam_loc, o_acc, total;
+  size_t zero, zero_bytes, counts, cursor, nitems, offs, list, items, part;   // chunk-major path
 };
+// Prefill route attention chunk-major over the whole sequence (chunk_major.cuh): fast shapes
+// whose selections fit the entry encoding (row << 6 | slot).
+bool cm_path_ok(const rdl_dims* dm, rdl_dtype t) {
+  return fast_attn(dm, t) && dm->L / S <= CM_MAXC && dm->K <= 64 && dm->Lq < (1 << 25);
+}
+// The row-tile kernel (chunk_tc.cuh) shares each chunk's K/V among the rows of a 45-row tile that
+// selected it; when those buckets average fewer than 4 rows (long sequences: about 45 K / C)
+// the chunk-major path, which gathers every row of a chunk, takes over.
+bool use_chunk_major(const rdl_dims* dm, rdl_dtype t) {
+  return cm_path_ok(dm, t) && (double)CT_TQ * dm->K < 4.0 * (dm->L / S);
+}
+size_t cm_max_items(const rdl_dims* dm) {
+  const size_t bg = (size_t)dm->B * dm->Hkv, C = dm->L / S;
+  return (bg * dm->Lq * dm->K + CM_IT - 1) / CM_IT + bg * C;
+}
 AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
   AttnWs w{};
   if (!fast_attn(dm, t)) return w;
@@ -211,7 +244,7 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
     // [B, Lq, Hq, d] and its (max, sum) [B, Lq, Hq]
     const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
     size_t off = 0;
-    w.o_acc = off;   off += align256(sizeof(float) * rows * dm->K * dm->d);
+    w.o_acc = off;   off += align256(sizeof(__half) * rows * dm->K * dm->d);
     w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d);
     w.lam_loc = off; off += align256(sizeof(float2) * rows);
     w.total = off;
@@ -223,11 +256,32 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
   w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d * nsw);
   w.lam_loc = off; off += align256(sizeof(float) * rows * nsw);
   w.o_acc = off;
+  if (use_chunk_major(dm, t)) {
+    // bucket counts, cursors and the item count (zeroed by one memset), bucket offsets, the
+    // bucketed selections, the work items and the fp16 chunk outputs [B*Hkv, Lq, K, G, d]
+    const size_t bg = (size_t)dm->B * dm->Hkv, C = dm->L / S, G = dm->Hq / dm->Hkv;
+    w.zero = off;
+    w.counts = off;  off += sizeof(int) * bg * C;
+    w.cursor = off;  off += sizeof(int) * bg * C;
+    w.nitems = off;  off += sizeof(int);
+    w.zero_bytes = off - w.zero;
+    off = align256(off);
+    w.offs = off;    off += align256(sizeof(int) * bg * C);
+    w.list = off;    off += align256(sizeof(int) * bg * dm->Lq * dm->K);
+    w.items = off;   off += align256(sizeof(CmItem) * cm_max_items(dm));
+    w.part = off;    off += align256(sizeof(__half) * bg * dm->Lq * dm->K * G * dm->d);
+    w.total = off;
+    return w;
+  }
   const int ns = attn_splits(dm);
   if (ns > 1) off += align256(sizeof(float) * rows * dm->d * ns);
   w.total = off;
   return w;
 }
+
+rdl_status attn_chunk_major(const void* q, const int32_t* q_pos, const void* k, const void* v, const int32_t* idx,
+                            const float* z_sel, const rdl_dims* dm, void* o, float* lse, void* workspace,
+                            cudaStream_t st);
 
 // Sliding-window workspace: key-split partials when the row count is small (else none).
 size_t swa_ws(const rdl_dims* dm, rdl_dtype t) {
@@ -340,7 +394,7 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
                        cudaStream_t st) {
   const AttnWs wl = attn_ws(dm, RDL_BF16);
   char* ws = static_cast<char*>(workspace);
-  float* o_part = reinterpret_cast<float*>(ws + wl.o_acc);
+  __half* o_part = reinterpret_cast<__half*>(ws + wl.o_acc);
   float* ow = reinterpret_cast<float*>(ws + wl.o_loc);
   float2* ml = reinterpret_cast<float2*>(ws + wl.lam_loc);
   const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
@@ -380,7 +434,7 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
     return RDL_ERR_CUDA;
   if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), dec::COMB_SPREAD_SMEM, st,
                  q_pos, idx, z_sel,
-                 (const float*)o_part, (const float*)ow, (const float2*)ml, dm->B, dm->L, dm->Lq, dm->Hq,
+                 (const __half*)o_part, (const float*)ow, (const float2*)ml, dm->B, dm->L, dm->Lq, dm->Hq,
                  dm->Hkv, dm->K, dm->w, dm->flags, static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
     return RDL_ERR_CUDA;
   return RDL_OK;
@@ -432,12 +486,33 @@ rdl_status score_fast(const void* q, const int32_t* q_pos, const void* x, const 
         !make_tmap_bf16_nd(&spmap, reinterpret_cast<const char*>(sb) + 512, 3, pd, ps, pb) ||
         !make_tmap_bf16_nd(&tmap, tt, 3, td, ts, tb))
       return RDL_ERR_CUDA;
-    if (cudaFuncSetAttribute(zeta_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ZT_SMEM) != cudaSuccess)
-      return RDL_ERR_CUDA;
     dim3 grid((C + ZT_CH - 1) / ZT_CH, (dm->Lq + ZT_ROWS - 1) / ZT_ROWS, dm->B * dm->Hkv);
+    if (fused_score(dm, RDL_BF16)) {
+      // group maxima only, the top-K on them, then the products again for the selected
+      // chunks' per-head scores: no per-head score buffer
+      if (cudaFuncSetAttribute(zeta_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ZT_SMEM) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(zeta_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, ZT_SMEM) != cudaSuccess)
+        return RDL_ERR_CUDA;
+      count_launch();
+      zeta_tc_kernel<1><<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
+                                                           dm->Hq, dm->Hkv, dm->w, dm->lambda, nullptr, zeta, nullptr,
+                                                           dm->K, nullptr);
+      if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
+      rdl_status s2 = launch_topk(zeta, nullptr, q_pos, dm, idx, z_sel, st);
+      if (s2 != RDL_OK) return s2;
+      count_launch();
+      zeta_tc_kernel<2><<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
+                                                           dm->Hq, dm->Hkv, dm->w, dm->lambda, nullptr, nullptr, idx,
+                                                           dm->K, z_sel);
+      return cuda_status(cudaGetLastError());
+    }
+    if (cudaFuncSetAttribute(zeta_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, ZT_SMEM) != cudaSuccess)
+      return RDL_ERR_CUDA;
     count_launch();
-    zeta_tc_kernel<<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
-                                                      dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta);
+    zeta_tc_kernel<0><<<grid, ZT_THREADS, ZT_SMEM, st>>>(qmap, smap, spmap, tmap, q_pos, entropy, dm->Lq, dm->L,
+                                                         dm->Hq, dm->Hkv, dm->w, dm->lambda, z_all, zeta, nullptr,
+                                                         dm->K, nullptr);
   }
   if (cudaGetLastError() != cudaSuccess) return RDL_ERR_CUDA;
   return launch_topk(zeta, z_all, q_pos, dm, idx, z_sel, st);
@@ -568,6 +643,54 @@ rdl_status launch_window_mma(const void* q, const int32_t* q_pos, const void* k,
   return cuda_status(cudaGetLastError());
 }
 
+rdl_status attn_chunk_major(const void* q, const int32_t* q_pos, const void* k, const void* v, const int32_t* idx,
+                            const float* z_sel, const rdl_dims* dm, void* o, float* lse, void* workspace,
+                            cudaStream_t st) {
+  const AttnWs wl = attn_ws(dm, RDL_BF16);
+  char* ws = static_cast<char*>(workspace);
+  float* o_loc = reinterpret_cast<float*>(ws + wl.o_loc);
+  float* lam_loc = reinterpret_cast<float*>(ws + wl.lam_loc);
+  int* counts = reinterpret_cast<int*>(ws + wl.counts);
+  int* cursor = reinterpret_cast<int*>(ws + wl.cursor);
+  int* nitems = reinterpret_cast<int*>(ws + wl.nitems);
+  int* offs = reinterpret_cast<int*>(ws + wl.offs);
+  int* list = reinterpret_cast<int*>(ws + wl.list);
+  CmItem* items = reinterpret_cast<CmItem*>(ws + wl.items);
+  __half* part = reinterpret_cast<__half*>(ws + wl.part);
+  const int C = dm->L / S, BG = dm->B * dm->Hkv;
+  // the local window: normalised output and log-sum-exp per (row, head)
+  const int nsw = window_splits(dm);
+  rdl_status s = launch_window_mma<1>(q, q_pos, k, v, dm, nullptr, nullptr, o_loc, lam_loc, nsw, st);
+  if (s != RDL_OK) return s;
+  // buckets of selections per (batch, group, chunk) and the work items
+  if (cudaMemsetAsync(ws + wl.zero, 0, wl.zero_bytes, st) != cudaSuccess) return RDL_ERR_CUDA;
+  const dim3 bgrid((dm->Lq + CM_ROWS - 1) / CM_ROWS, BG);
+  if (cudaFuncSetAttribute(cm_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C * 4) != cudaSuccess ||
+      cudaFuncSetAttribute(cm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * C * 4) != cudaSuccess ||
+      cudaFuncSetAttribute(cm_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CM_SMEM) != cudaSuccess)
+    return RDL_ERR_CUDA;
+  count_launch(5);
+  cm_count_kernel<<<bgrid, 512, C * 4, st>>>(idx, q_pos, dm->Lq, dm->L, dm->Hkv, dm->K, dm->w, dm->flags, counts);
+  cm_scan_kernel<<<BG, 1024, 0, st>>>(counts, C, offs, nitems, items);
+  cm_scatter_kernel<<<bgrid, 512, 2 * C * 4, st>>>(idx, q_pos, dm->Lq, dm->L, dm->Hkv, dm->K, dm->w, dm->flags, offs,
+                                                  cursor, list);
+  // chunk passes: persistent CTAs, one per SM
+  CUtensorMap kmap, vmap, qmap;
+  const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
+  if (!make_tmap_kv_halves(&kmap, k, kvrows) || !make_tmap_kv_halves(&vmap, v, kvrows) ||
+      !make_tmap_q_run(&qmap, q, (unsigned long long)dm->B * dm->Lq, (unsigned)dm->Hq, 1))
+    return RDL_ERR_CUDA;
+  const size_t mi = cm_max_items(dm);
+  const int grid = (int)(mi < (size_t)kSMs ? mi : (size_t)kSMs);
+  cm_attn_kernel<<<grid, CM_THREADS, CM_SMEM, st>>>(kmap, vmap, qmap, items, nitems,
+                                                   list, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K, dm->flags, part);
+  const long long n = (long long)dm->B * dm->Lq * dm->Hq;
+  cm_combine_kernel<<<(unsigned)((n + 7) / 8), 256, 0, st>>>(q_pos, idx, z_sel, part, o_loc, lam_loc, nsw, dm->B, dm->L,
+                                                             dm->Lq, dm->Hq, dm->Hkv, dm->K, dm->w, dm->flags,
+                                                             static_cast<__nv_bfloat16*>(o), lse);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -679,6 +802,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
   if (ws_bytes < wl.total) return RDL_ERR_WORKSPACE;
   if (dec_attn_ok(dims, dtype) && dec_attn_stages(dims, dims->K) > 0)
     return attn_decode(q, q_pos, k, v, idx, z_sel, dims, o, lse, workspace, st);
+  if (use_chunk_major(dims, dtype)) return attn_chunk_major(q, q_pos, k, v, idx, z_sel, dims, o, lse, workspace, st);
   char* ws = static_cast<char*>(workspace);
   float* o_loc = reinterpret_cast<float*>(ws + wl.o_loc);
   float* lam_loc = reinterpret_cast<float*>(ws + wl.lam_loc);

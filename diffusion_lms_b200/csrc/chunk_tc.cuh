@@ -69,7 +69,7 @@ constexpr int CT_OFF_KV = 0;                                   // slot s: K at s
 constexpr int CT_OFF_A = CT_OFF_KV + CT_NSLOT * 32768;         // NA x 16 KB Q tiles
 constexpr int CT_OFF_P = CT_OFF_A + CT_NA * 16384;             // 2 x 8 KB P tiles
 constexpr int CT_OFF_BAR = CT_OFF_P + 2 * 8192;                // mbarriers
-constexpr int CT_NBAR = 2 * CT_NSLOT + 2 * CT_NA + 11;
+constexpr int CT_NBAR = 2 * CT_NSLOT + 2 * CT_NA + 12;
 constexpr int CT_OFF_MISC = CT_OFF_BAR + 256;                  // tmem base, abort, nunion
 constexpr int CT_OFF_MASK = CT_OFF_MISC + 128;                 // row masks [MAXC] u64
 constexpr int CT_OFF_OFS = CT_OFF_MASK + CT_MAXC * 8;          // bucket offsets [MAXC] int
@@ -104,7 +104,9 @@ struct CtBars {
   uint64_t* tfull;   // T ready (commit)
   uint64_t* tempty;  // T added into the home columns (8 arrivals)
   uint64_t* done;    // [2] every MMA of the S / PV issuer complete (before TMEM is freed)
+  uint64_t* never;   // nothing arrives on it (RDL_FLAG_WAIT_TEST)
 };
+constexpr unsigned CT_TEST_POLLS = 1u << 12;   // bound of the RDL_FLAG_WAIT_TEST wait
 
 // bounded wait that also gives up as soon as another role has aborted
 __device__ __forceinline__ bool ct_wait(uint64_t* bar, unsigned parity, volatile int* abort_flag) {
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CT_OFF_BAR);
   uint64_t* b2 = bars + 2 * CT_NSLOT + 2 * CT_NA;
   CtBars B{bars, bars + CT_NSLOT, bars + 2 * CT_NSLOT, bars + 2 * CT_NSLOT + CT_NA,
-           b2, b2 + 2, b2 + 3, b2 + 5, b2 + 7, b2 + 8, b2 + 9};
+           b2, b2 + 2, b2 + 3, b2 + 5, b2 + 7, b2 + 8, b2 + 9, b2 + 11};
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + CT_OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CT_OFF_MISC + 4);
   int* nunion_s = reinterpret_cast<int*>(sm + CT_OFF_MISC + 8);
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     tc::mbar_init(B.sempty, 4);
     tc::mbar_init(B.tfull, 1);
     tc::mbar_init(B.tempty, 8);
+    tc::mbar_init(B.never, 1);
     tc::mbar_fence_init();
     *abort_flag = 0;
   }
@@ -381,6 +384,18 @@ __global__ void __launch_bounds__(CT_THREADS, 1) chunk_tc_kernel(
     for (int u = 0; u < U && ok; ++u) {
       const int n = __shfl_sync(0xffffffffu, (int)(uni[u] >> 24), 0), slot = u % CT_NSLOT;
       if (!__all_sync(0xffffffffu, ct_wait(&B.full[slot], (u / CT_NSLOT) & 1, abort_flag))) break;
+      if ((flags & RDL_FLAG_WAIT_TEST) && u == 0) {
+        // a wait on a barrier nothing arrives on runs out: the failure path of every wait
+        bool got = false;
+        for (unsigned x = 0; x < CT_TEST_POLLS && !got; ++x) got = tc::mbar_try_wait(B.never, 0);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) {
+            record_status(RDL_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+      }
       const uint64_t dk = dK0 + (uint64_t)((slot * 32768) >> 4);
       for (int p0 = 0; p0 < n; p0 += CT_QP, ++k) {
         const int ab = k % CT_NA, sb = k & 1;

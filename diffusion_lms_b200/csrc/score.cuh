@@ -408,11 +408,13 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
   for (int k = taken + lane; k < K; k += 32) irow[k] = -1;
   __syncwarp();
   const int nsel = taken < K ? taken : K;
+  // per-head scores of the selection (without z_all they come later, from the scorer's second
+  // pass over the selected chunks; every slot starts at -inf)
   for (int e = lane; e < K * G; e += 32) {
     const int k = e % K, hl = e / K, h = g * G + hl;
     const int c = (k < nsel) ? irow[k] : -1;
     z_sel[((size_t)(b * Hq + h) * Lq + i) * K + k] =
-        (c >= 0) ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
+        (c >= 0 && z_all) ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
   }
 }
 
@@ -608,7 +610,7 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
     const int c = k < nsel ? sel_s[k] : -1;
     if (hl == 0) irow[k] = c;
     z_sel[((size_t)(b * Hq + h) * Lq + i) * K + k] =
-        c >= 0 ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
+        (c >= 0 && z_all) ? z_all[((size_t)(b * Hq + h) * Lq + i) * C + c] : -INFINITY;
   }
 }
 

@@ -34,11 +34,17 @@ constexpr int ZT_OFF_P = ZT_OFF_H + 8 * ZT_CH * 4;        // positions [128] int
 constexpr int ZT_SMEM = ZT_OFF_P + ZT_ROWS * 4 + 1024;    // + alignment slack
 static_assert(ZT_SMEM <= 227 * 1024, "shared memory");
 
+// MODE 0: writes every per-head score (z_all) and the group maximum (zeta);
+// MODE 1: writes the group maximum only;
+// MODE 2: given the selection idx (ascending per row and group), writes the per-head scores of
+//         the selected chunks that fall in the CTA's chunk tile into z_sel.
+template <int MODE>
 __global__ void __launch_bounds__(ZT_THREADS, 1)
     zeta_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap smap,
                    const __grid_constant__ CUtensorMap spmap, const __grid_constant__ CUtensorMap tmap,
                    const int32_t* __restrict__ q_pos, const float* __restrict__ entropy, int Lq, int L, int Hq,
-                   int Hkv, int w, float lambda, float* __restrict__ z_all, float* __restrict__ zeta) {
+                   int Hkv, int w, float lambda, float* __restrict__ z_all, float* __restrict__ zeta,
+                   const int32_t* __restrict__ idx, int K, float* __restrict__ z_sel) {
   constexpr int D = 128;
   extern __shared__ unsigned char zt_raw[];
   unsigned char* sm = zt_raw + ((1024u - (smem_u32(zt_raw) & 1023u)) & 1023u);
@@ -175,6 +181,32 @@ __global__ void __launch_bounds__(ZT_THREADS, 1)
     for (int e = 0; e < 32; ++e) zmax[e] = -INFINITY;
     const bool vec = (C & 3) == 0 && cb + 32 <= C;
     bool ok = true;
+    // MODE 2: the row's selection as a mask over chunks cb .. cb + 31 (bit e: chunk cb + e is
+    // selected) and k0, the number of selected chunks below cb, so that chunk cb + e sits in
+    // slot k0 + popc(sel & ((1 << e) - 1)) of the ascending list; the row's K indices are
+    // loaded at once (K <= 64)
+    uint32_t sel = 0u;
+    int k0 = 0;
+    if (MODE == 2 && i < Lq) {
+      const int32_t* irow = idx + ((size_t)bg * Lq + i) * K;
+      int v[64];
+      if ((K & 3) == 0) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int4 q4 = 4 * u < K ? __ldg(reinterpret_cast<const int4*>(irow) + u) : make_int4(-1, -1, -1, -1);
+          v[4 * u] = q4.x; v[4 * u + 1] = q4.y; v[4 * u + 2] = q4.z; v[4 * u + 3] = q4.w;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 64; ++u) v[u] = u < K ? __ldg(irow + u) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 64; ++u) {
+        const int c = v[u];
+        if (c >= 0 && c < cb) ++k0;
+        if (c >= cb && c < cb + 32) sel |= 1u << (c - cb);
+      }
+    }
     for (int hl = 0; hl < G; ++hl) {
       const int hb = hl & 1;
       if (!wait_all(&afull[hb], (unsigned)(hl >> 1) & 1u)) { ok = false; break; }
@@ -194,7 +226,14 @@ __global__ void __launch_bounds__(ZT_THREADS, 1)
         z[e] = ((em >> e) & 1u) ? tau * (v1[e] + (v2[e] + v3[e])) - lambda * hrow[e] : -INFINITY;
         zmax[e] = fmaxf(zmax[e], z[e]);
       }
-      if (i < Lq) {
+      if (MODE == 2) {
+        if (sel) {
+          float* zs = z_sel + ((size_t)(b * Hq + g * G + hl) * Lq + i) * K + k0;
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if ((sel >> x) & 1u) zs[__popc(sel & ((1u << x) - 1u))] = z[x];
+        }
+      } else if (MODE == 0 && i < Lq) {
         float* zr = z_all + ((size_t)(b * Hq + g * G + hl) * Lq + i) * C + cb;
         if (vec) {
 #pragma unroll
@@ -206,7 +245,7 @@ __global__ void __launch_bounds__(ZT_THREADS, 1)
         }
       }
     }
-    if (ok && i < Lq) {
+    if (MODE != 2 && ok && i < Lq) {
       float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C + cb;
       if (vec) {
 #pragma unroll
@@ -225,5 +264,9 @@ __global__ void __launch_bounds__(ZT_THREADS, 1)
   tc::tc_fence_after();
   if (warp == 0) tc::tmem_dealloc(tbase, 512);
 }
+
+}  // namespace rdl
+
+namespace rdl {
 
 }  // namespace rdl

@@ -26,7 +26,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_
 ERR_SCRATCH_LIMIT = -7
 NOALLOC_SCRATCH_BYTES = 32 << 20
 BF16, F32 = 0, 1
-FLAG_MEAN_SUMMARY, FLAG_CHECKS, FLAG_SPLIT_SUMMARY = 0x1, 0x2, 0x4
+FLAG_MEAN_SUMMARY, FLAG_CHECKS, FLAG_SPLIT_SUMMARY, FLAG_WAIT_TEST = 0x1, 0x2, 0x4, 0x8
 WS_SCORE, WS_ATTN, WS_SWA = 0, 1, 2
 CHUNK = 64
 

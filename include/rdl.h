@@ -73,6 +73,13 @@ typedef enum { RDL_BF16 = 0, RDL_F32 = 1 } rdl_dtype;
  * it for decode-block shapes (bf16, d = 128, at most 64 rows) and returns
  * RDL_ERR_UNSUPPORTED otherwise. */
 #define RDL_FLAG_SPLIT_SUMMARY 0x4
+/* Test only: the failure path of a bounded wait.  With this flag the prefill selected-chunk
+ * kernel of rdl_route_attn (either of its two forms) waits, with a short limit, on a barrier
+ * nothing arrives on, once its first K/V slab and query loads are in flight.  The wait runs out: the
+ * kernel records RDL_ERR_TIMEOUT, every role stops, the copies and MMAs in flight drain, tensor
+ * memory is freed and the kernel returns; the call's outputs are then not valid.  Nothing
+ * faults and the context stays usable (the next call without the flag computes normally). */
+#define RDL_FLAG_WAIT_TEST 0x8
 
 #define RDL_CHUNK 64
 
@@ -176,7 +183,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * that loads the library, until the process exits.  A call whose
  * rdl_workspace_bytes(RDL_WS_ATTN, dims, dtype) exceeds it returns RDL_ERR_SCRATCH_LIMIT
  * and launches nothing (a 32-query decode block over 28 heads with K = 32 and a +-256 window
- * needs about 14.5 MiB).
+ * needs about 7.4 MiB).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture begins.  The
  * address is kept per device and context: after cudaDeviceReset the next call on that

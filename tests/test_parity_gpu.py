@@ -221,6 +221,39 @@ def test_decode_device_checks_record_without_fault():
     assert torch.isfinite(out.o.float()).all()
 
 
+@pytest.mark.parametrize("L,K", [(2048, 4), (4096, 2)])
+def test_wait_timeout_returns_and_the_next_call_computes(L, K):
+    """Failure detection without a fault: with RDL_FLAG_WAIT_TEST the prefill selected-chunk
+    kernel waits, with a short limit, on a barrier nothing arrives on, once its first K/V slab
+    and query loads are in flight (row-tile form for L = 2048 with K = 4; chunk-major form for
+    L = 4096 with K = 2).  The call returns, the status word reads RDL_ERR_TIMEOUT (then
+    clears), and the next calls in the same process match the oracle."""
+    wl = W.make_inputs(small(L=L, Lq=L, Hq=8, Hkv=2, K=K, w=64), seed=35, n_needles=2)
+    inp = api.to_device(wl)
+    out = api.alloc_outputs(inp.dims, inp.dtype)
+    api.summary_pool(inp, out)
+    api.score_topk(inp, out)
+    torch.cuda.synchronize()
+    assert rdl.rdl_last_device_status() == rdl.OK
+    inp.dims.flags = rdl.FLAG_WAIT_TEST
+    api.route_attn(inp, out)
+    assert rdl.rdl_last_device_status() == rdl.ERR_TIMEOUT
+    assert rdl.rdl_last_device_status() == rdl.OK           # cleared on read
+    gpu = P.run_gpu(wl)
+    P.check_route_layer(wl, gpu, np.arange(0, L, 3))
+
+
+def test_chunk_major_prefill_rows():
+    """The chunk-major form of the selected-chunk attention (each chunk's rows gathered over
+    the whole sequence, fp16 chunk outputs, a separate combine) on a prefill whose chunk
+    buckets per 45-row tile would be small (8K rows, K = 2 of 128 chunks), every third row,
+    with a second batch element."""
+    wl = W.make_inputs(small(B=2, L=8192, Lq=8192, Hq=8, Hkv=2, K=2, w=64), seed=36, n_needles=4)
+    gpu = P.run_gpu(wl)
+    rows = np.unique(np.concatenate([np.arange(0, 8192, 3), np.arange(8100, 8192)]))
+    P.check_route_layer(wl, gpu, rows)
+
+
 def test_bitwise_repeatable():
     for dm, dec in ((small(), 0), (small(L=8192, Lq=32, K=32, w=256), 32)):
         wl = W.make_inputs(dm, seed=18, n_needles=4, decode_block=dec)
