@@ -195,7 +195,7 @@ def job_throughput(rows_per_rank: int, world: int, ms_max: float) -> float:
 # a share of the sampled rows.  Each worker receives the stored (bf16 bit) inputs it needs and
 # calls only oracle functions; the parent measures the wall time of both phases.
 
-MAX_ORACLE_WORKERS = 64
+MAX_ORACLE_WORKERS = 32
 _ORACLE_WL = {}
 
 
@@ -203,10 +203,13 @@ def oracle_workers() -> int:
     return max(1, min(os.cpu_count() or 1, MAX_ORACLE_WORKERS))
 
 
-def _oracle_init(arrays):
-    """Worker start-up: keep the workload's stored inputs (sent once per worker)."""
+def _oracle_init(maker, seed):
+    """Worker start-up: draw the workload's stored inputs from its seed (the same bits the
+    parent holds; the generator is deterministic)."""
+    from diffusion_lms_b200 import workloads as W
+    wl = getattr(W, maker)(seed=seed)
     _ORACLE_WL.clear()
-    _ORACLE_WL.update(arrays)
+    _ORACLE_WL.update({n: getattr(wl, n) for n in ("q", "q_mask", "k", "v", "x", "w_down", "w_up")})
 
 
 def _oracle_pool_heads(task):
@@ -242,13 +245,12 @@ def _oracle_rows(task):
 class OracleRunner:
     """Spawn-started worker pool timing the oracle on bounded samples of one workload."""
 
-    def __init__(self, wl, workers: int):
+    def __init__(self, wl, maker: str, seed: int, workers: int):
         import multiprocessing as mp
         self.wl = wl
         self.workers = workers
-        arrays = {n: getattr(wl, n) for n in ("q", "q_mask", "k", "v", "x", "w_down", "w_up")}
         self.pool = mp.get_context("spawn").Pool(workers, initializer=_oracle_init,
-                                                 initargs=(arrays,))
+                                                 initargs=(maker, seed))
 
     def close(self):
         self.pool.close()
@@ -284,8 +286,8 @@ def run_reference(args, rank):
     from diffusion_lms_b200 import workloads as W
     if rank != 0:
         return
-    wl = W.prefill_16k()
-    runner = OracleRunner(wl, oracle_workers())
+    wl = W.prefill_16k(seed=2)
+    runner = OracleRunner(wl, "prefill_16k", 2, oracle_workers())
     n = args.ref_rows if args.ref_rows > 0 else 16 * runner.workers
     for _ in range(args.warmup):
         runner.sample(max(runner.workers, n // 8))
@@ -636,7 +638,7 @@ def main():
     wl = W.prefill_16k(seed=rank_seed(2, rank))
     runner = None
     if rank == 0 and not args.no_cpu_baseline:
-        runner = OracleRunner(wl, oracle_workers())
+        runner = OracleRunner(wl, "prefill_16k", rank_seed(2, rank), oracle_workers())
 
     import torch
     import torch.distributed as dist
