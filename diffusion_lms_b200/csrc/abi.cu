@@ -244,7 +244,7 @@ AttnWs attn_ws(const rdl_dims* dm, rdl_dtype t) {
     // [B, Lq, Hq, d] and its (max, sum) [B, Lq, Hq]
     const size_t rows = (size_t)dm->B * dm->Lq * dm->Hq;
     size_t off = 0;
-    w.o_acc = off;   off += align256(sizeof(__half) * rows * dm->K * dm->d);
+    w.o_acc = off;   off += align256(sizeof(float) * rows * dm->K * dm->d);
     w.o_loc = off;   off += align256(sizeof(float) * rows * dm->d);
     w.lam_loc = off; off += align256(sizeof(float2) * rows);
     w.total = off;
@@ -394,7 +394,7 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
                        cudaStream_t st) {
   const AttnWs wl = attn_ws(dm, RDL_BF16);
   char* ws = static_cast<char*>(workspace);
-  __half* o_part = reinterpret_cast<__half*>(ws + wl.o_acc);
+  float* o_part = reinterpret_cast<float*>(ws + wl.o_acc);
   float* ow = reinterpret_cast<float*>(ws + wl.o_loc);
   float2* ml = reinterpret_cast<float2*>(ws + wl.lam_loc);
   const unsigned long long kvrows = (unsigned long long)dm->B * dm->Hkv * dm->L;
@@ -434,7 +434,7 @@ rdl_status attn_decode(const void* q, const int32_t* q_pos, const void* k, const
     return RDL_ERR_CUDA;
   if (launch_pdl(dec::dec_comb_kernel<true>, dim3((unsigned)((items + 7) / 8)), dim3(256), dec::COMB_SPREAD_SMEM, st,
                  q_pos, idx, z_sel,
-                 (const __half*)o_part, (const float*)ow, (const float2*)ml, dm->B, dm->L, dm->Lq, dm->Hq,
+                 (const float*)o_part, (const float*)ow, (const float2*)ml, dm->B, dm->L, dm->Lq, dm->Hq,
                  dm->Hkv, dm->K, dm->w, dm->flags, static_cast<__nv_bfloat16*>(o), lse) != cudaSuccess)
     return RDL_ERR_CUDA;
   return RDL_OK;

@@ -766,8 +766,7 @@ __global__ void __launch_bounds__(DK_THREADS) dec_topk_kernel(const float* __res
 // as much as many sparse ones.  A CTA streams its chunks' K/V once through a TMA ring;
 // each consumer warp computes two tasks of a slab at once (M = 16 = two rows x 8 head
 // slots) with the probabilities kept in registers (no shared-memory round trip), and
-// writes o_part[b,i,g,k] = the softmax-normalised output of chunk idx[k] (fp16: a convex
-// combination of the chunk's values, stored once and read once by the combine).
+// writes o_part[b,i,g,k] = the softmax-normalised output of chunk idx[k].
 // dec_comb_kernel merges a row's window part and chunk outputs in a fixed order.
 // =====================================================================================
 constexpr int AT_CONS = 15;
@@ -872,7 +871,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     const __nv_bfloat16* __restrict__ kv_base_k, const __nv_bfloat16* __restrict__ kv_base_v,
                     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ q_pos,
                     const int32_t* __restrict__ idx, int L, int Lq, int Hq, int Hkv, int K, int w, int flags,
-                    int R, int stages, float sl2, __half* __restrict__ o_part) {
+                    int R, int stages, float sl2, float* __restrict__ o_part) {
   constexpr int D = 128;
   extern __shared__ unsigned char at_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(at_raw) + 1023) & ~uintptr_t(1023));
@@ -956,16 +955,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   }
   __syncthreads();
-  // Every needed slab is pulled into L2 once, by the CTA j == c % R, while the work partition
-  // below is computed; the owner's TMA loads then find it in L2 or in flight.
-  if (ROUTE) {
-    for (int c = j + R * tid; c < C; c += R * AT_THREADS) {
-      if (hist[c] == 0) continue;
-      const size_t off = (kvrow0 + (size_t)S * c) * D;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(kv_base_k + off), "r"(S * D * 2) : "memory");
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(kv_base_v + off), "r"(S * D * 2) : "memory");
-    }
-  }
   // One scan gives both prefixes in chunk order: pre[c] = first list position of slab c's
   // tasks, and the work prefix, work of slab c = its row pairs plus one slab load (weighted
   // AT_SLAB_WORK pairs).  Slab c belongs to CTA floor((work prefix(c) + work(c) / 2) * R /
@@ -1133,8 +1122,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         pa[kk][2] = pack_bf16(sc[2 * kk + 1][0] * fA, sc[2 * kk + 1][1] * fA);
         pa[kk][3] = pack_bf16(sc[2 * kk + 1][2] * fB, sc[2 * kk + 1][3] * fB);
       }
-      __half* dstA = nullptr;
-      __half* dstB = nullptr;
+      float* dstA = nullptr;
+      float* dstB = nullptr;
       {
         const int slotA = tA & 127, slotB = tB & 127;
         const size_t rgA = (size_t)(b * Lq + iA) * Hkv + g, rgB = (size_t)(b * Lq + iB) * Hkv + g;
@@ -1164,12 +1153,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (dstA) {
 #pragma unroll
           for (int nt = 0; nt < 8; ++nt)
-            *reinterpret_cast<__half2*>(dstA + 64 * half + 8 * nt + 2 * tq) = __floats2half2_rn(oc[nt][0], oc[nt][1]);
+            *reinterpret_cast<float2*>(dstA + 64 * half + 8 * nt + 2 * tq) = make_float2(oc[nt][0], oc[nt][1]);
         }
         if (dstB) {
 #pragma unroll
           for (int nt = 0; nt < 8; ++nt)
-            *reinterpret_cast<__half2*>(dstB + 64 * half + 8 * nt + 2 * tq) = __floats2half2_rn(oc[nt][2], oc[nt][3]);
+            *reinterpret_cast<float2*>(dstB + 64 * half + 8 * nt + 2 * tq) = make_float2(oc[nt][2], oc[nt][3]);
         }
       }
     }
@@ -1450,18 +1439,11 @@ __global__ void __launch_bounds__(SW_WARPS * 32, 1)
 // harmless).
 // =====================================================================================
 constexpr int COMB_SPREAD_SMEM = 120 * 1024;   // dynamic shared memory requested (unused)
-// four consecutive fp16 values (8-byte aligned) as fp32
-__device__ __forceinline__ float4 ld_half4(const __half* p) {
-  const uint2 r = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
 template <bool ROUTE>
 __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict__ q_pos,
                                                        const int32_t* __restrict__ idx,
                                                        const float* __restrict__ z_sel,
-                                                       const __half* __restrict__ o_part,
+                                                       const float* __restrict__ o_part,
                                                        const float* __restrict__ ow,
                                                        const float2* __restrict__ ml, int B, int L, int Lq,
                                                        int Hq, int Hkv, int K, int w, int flags,
@@ -1492,7 +1474,7 @@ __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict
   }
   int ck[2] = {-1, -1};
   float zr[2] = {-INFINITY, -INFINITY};
-  const __half* pbase = o_part + (rg * K * G + hl) * D + 4 * lane;
+  const float* pbase = o_part + (rg * K * G + hl) * D + 4 * lane;
   float4 v0[16];
   if (ROUTE) {
     const int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
@@ -1507,7 +1489,7 @@ __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u)
-      v0[u] = u < K ? ld_half4(pbase + (size_t)u * G * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v0[u] = u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)u * G * D) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   float zk[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -1533,7 +1515,7 @@ __global__ void __launch_bounds__(256) dec_comb_kernel(const int32_t* __restrict
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         v[u] = k0 == 0 ? v0[u]
-                       : (k0 + u < K ? ld_half4(pbase + (size_t)(k0 + u) * G * D)
+                       : (k0 + u < K ? *reinterpret_cast<const float4*>(pbase + (size_t)(k0 + u) * G * D)
                                      : make_float4(0.f, 0.f, 0.f, 0.f));
 #pragma unroll
       for (int u = 0; u < 16; ++u) {

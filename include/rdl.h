@@ -183,7 +183,7 @@ rdl_status rdl_route_attn(const void* q, const int32_t* q_pos, const void* k, co
  * that loads the library, until the process exits.  A call whose
  * rdl_workspace_bytes(RDL_WS_ATTN, dims, dtype) exceeds it returns RDL_ERR_SCRATCH_LIMIT
  * and launches nothing (a 32-query decode block over 28 heads with K = 32 and a +-256 window
- * needs about 7.4 MiB).
+ * needs about 14.5 MiB).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture begins.  The
  * address is kept per device and context: after cudaDeviceReset the next call on that
