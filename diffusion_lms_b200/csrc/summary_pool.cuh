@@ -4,10 +4,15 @@
 // pooling weights is the second routing signal).
 //
 // One CTA per (chunk c, KV head g, batch b): the chunk's 63 content keys (and values)
-// are read from HBM once, staged in shared memory as fp32, and reused by every query
-// head of the group.  The kernel streams K/V once, so it is HBM-bound.
+// are read from HBM once into shared memory and reused by every query head of the group.
+// The pass streams K/V once, so it is HBM-bound.  bf16 inputs take summary_pool_bulk_kernel
+// (one bulk copy per slab, bf16 in shared memory, 32 KB per CTA, so several CTAs per SM keep
+// their copies in flight together); fp32 inputs, or mask-query strides that do not keep a
+// lane's elements aligned, take summary_pool_kernel (fp32 staging).
 #pragma once
+#include <type_traits>
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace rdl {
 
@@ -114,12 +119,194 @@ __global__ void __launch_bounds__(256) summary_pool_kernel(
   }
 }
 
+// E consecutive bf16 values (E = 2 or 4, 4- or 8-byte aligned) to / from fp32
+template <int E>
+__device__ __forceinline__ void ld_bf16_vec(const __nv_bfloat16* p, float* f) {
+  static_assert(E == 2 || E == 4, "two or four elements");
+  if constexpr (E == 4) {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    f[0] = a.x; f[1] = a.y; f[2] = c.x; f[3] = c.y;
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    f[0] = a.x; f[1] = a.y;
+  }
+}
+template <int E>
+__device__ __forceinline__ void st_bf16_vec(__nv_bfloat16* p, const float* f) {
+  static_assert(E == 2 || E == 4, "two or four elements");
+  const __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
+  if constexpr (E == 4) {
+    const __nv_bfloat162 c = __floats2bfloat162_rn(f[2], f[3]);
+    uint2 r;
+    r.x = *reinterpret_cast<const uint32_t*>(&a);
+    r.y = *reinterpret_cast<const uint32_t*>(&c);
+    *reinterpret_cast<uint2*>(p) = r;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(p) = a;
+  }
+}
+// One halving exchange of the reduce-scatter: p[0 .. 2 DIST) -> p[0 .. DIST), keeping the
+// half whose key bit DIST equals the lane's bit DIST and adding the partner's share of it.
+template <int DIST>
+__device__ __forceinline__ void rs_step(float* p, int lane) {
+  const bool upper = (lane & DIST) != 0;
+#pragma unroll
+  for (int t = 0; t < DIST; ++t) {
+    const float send = upper ? p[t] : p[DIST + t];
+    const float keep = upper ? p[DIST + t] : p[t];
+    p[t] = keep + __shfl_xor_sync(0xffffffffu, send, DIST);
+  }
+}
+
+// bf16 inputs: the chunk's 63 content keys (and values) arrive in shared memory by one bulk
+// copy each (16128 contiguous bytes of the [B, Hkv, L, d] cache) and stay bf16, so a CTA
+// holds 32 KB and several CTAs share an SM with their copies in flight at once.  Warp hl
+// takes head hl of the group; lane l owns the E = d/32 consecutive elements [E l, E l + E)
+// of every row (conflict-free row reads).  The 63 logits: per 32-key half, every lane forms
+// its partial dot products with its E elements, and a reduce-scatter over the warp (halving
+// exchanges at lane distances 16, 8, 4, 2, 1) leaves lane l the full logit of key l of the
+// half.  Softmax, entropy and the weighted sums then follow as in the fp32 kernel above.
+template <int D>
+__global__ void __launch_bounds__(256) summary_pool_bulk_kernel(
+    const __nv_bfloat16* __restrict__ q_mask, long long q_chunk_stride, long long q_batch_stride,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int L, int Hq, int Hkv,
+    int flags, float* __restrict__ summary, float* __restrict__ entropy, __nv_bfloat16* __restrict__ o_mask) {
+  constexpr int E = D / 32;                       // elements per lane
+  constexpr unsigned ROW_BYTES = CONTENT * D * 2;  // one slab of content rows (multiple of 16)
+  extern __shared__ __align__(128) unsigned char sp_raw[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(sp_raw);
+  __nv_bfloat16* Vs = Ks + CONTENT * D;
+  __shared__ __align__(8) uint64_t bar;
+
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t kv_base = ((size_t)(b * Hkv + g) * L + (size_t)c * S) * D;
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::mbar_fence_init();
+    tc::mbar_arrive_expect_tx(&bar, v ? 2 * ROW_BYTES : ROW_BYTES);
+    tc::bulk_load(Ks, k + kv_base, ROW_BYTES, &bar);
+    if (v) tc::bulk_load(Vs, v + kv_base, ROW_BYTES, &bar);
+  }
+  __syncthreads();
+
+  const float tau = rsqrtf((float)D);
+  const bool mean = (flags & RDL_FLAG_MEAN_SUMMARY) != 0;
+  const bool has1 = lane + 32 < CONTENT;
+  bool landed = false;
+  for (int hl = warp; hl < G; hl += blockDim.x / 32) {
+    const int h = g * G + hl;
+    const __nv_bfloat16* qrow = q_mask + (size_t)b * q_batch_stride + (size_t)c * q_chunk_stride + (size_t)h * D;
+    float qv[E];
+    ld_bf16_vec<E>(qrow + E * lane, qv);
+    if (!landed) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bar, 0))) return;   // bounded; status recorded
+      landed = true;
+    }
+    float l0 = 0.f, l1 = 0.f;
+    if (!mean) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float p[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int key = 32 * half + j;
+          float acc = 0.f;
+          if (key < CONTENT) {
+            float kv[E];
+            ld_bf16_vec<E>(Ks + key * D + E * lane, kv);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc = fmaf(qv[e], kv[e], acc);
+          }
+          p[j] = acc;
+        }
+        // reduce-scatter: after the exchange at distance s a lane keeps the values whose key
+        // bit s equals its own lane bit s; at the end lane l holds key l of the half
+        rs_step<16>(p, lane);
+        rs_step<8>(p, lane);
+        rs_step<4>(p, lane);
+        rs_step<2>(p, lane);
+        rs_step<1>(p, lane);
+        if (half == 0) l0 = p[0] * tau; else l1 = p[0] * tau;
+      }
+      if (!has1) l1 = -INFINITY;
+    } else {
+      l1 = has1 ? 0.f : -INFINITY;
+    }
+    const float m = warp_max(fmaxf(l0, l1));
+    const float e0 = expf(l0 - m), e1 = has1 ? expf(l1 - m) : 0.f;
+    const float z = warp_sum(e0 + e1);
+    const float inv = 1.f / z;
+    const float a0 = e0 * inv, a1 = e1 * inv;
+    const float sal = warp_sum(a0 * (l0 - m) + (has1 ? a1 * (l1 - m) : 0.f));
+    const float H = logf(z) - sal;
+
+    float sacc[E], oacc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sacc[e] = oacc[e] = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < CONTENT; ++j) {
+      const float aj = __shfl_sync(0xffffffffu, j < 32 ? a0 : a1, j & 31);
+      float kv[E];
+      ld_bf16_vec<E>(Ks + j * D + E * lane, kv);
+#pragma unroll
+      for (int e = 0; e < E; ++e) sacc[e] = fmaf(aj, kv[e], sacc[e]);
+      if (v) {
+        ld_bf16_vec<E>(Vs + j * D + E * lane, kv);
+#pragma unroll
+        for (int e = 0; e < E; ++e) oacc[e] = fmaf(aj, kv[e], oacc[e]);
+      }
+    }
+    float* srow = summary + ((size_t)(b * Hq + h) * C + c) * D;
+    if (flags & RDL_FLAG_SPLIT_SUMMARY) {
+      // the same 4D bytes as D bf16 hi terms, then D bf16 lo terms (s = hi + lo)
+      __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(srow);
+      float hv[E], lv[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(sacc[e]);
+        hv[e] = __bfloat162float(hi);
+        lv[e] = sacc[e] - hv[e];
+      }
+      st_bf16_vec<E>(hrow + E * lane, hv);
+      st_bf16_vec<E>(hrow + D + E * lane, lv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) srow[E * lane + e] = sacc[e];
+    }
+    if (lane == 0) entropy[(size_t)(b * Hq + h) * C + c] = H;
+    if (o_mask && v) {
+      __nv_bfloat16* orow = o_mask + (size_t)b * q_batch_stride + (size_t)c * q_chunk_stride + (size_t)h * D;
+      st_bf16_vec<E>(orow + E * lane, oacc);
+    }
+  }
+}
+
 template <typename T, int D>
 cudaError_t launch_summary_pool(const void* q_mask, long long qcs, long long qbs, const void* k,
                                 const void* v, const rdl_dims& dm, float* summary, float* entropy,
                                 void* o_mask, cudaStream_t st) {
   const int C = dm.L / S;
   const bool with_v = v != nullptr && o_mask != nullptr;
+  // the bulk kernel reads and writes a lane's D/32 mask-query elements as one vector: the
+  // strides must keep every mask row aligned to it
+  constexpr long long kVec = D / 32;
+  if (std::is_same<T, __nv_bfloat16>::value && qcs % kVec == 0 && qbs % kVec == 0) {
+    const size_t smem = (size_t)CONTENT * D * 2 * (with_v ? 2 : 1);
+    auto kern = summary_pool_bulk_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(C, dm.Hkv, dm.B);
+    count_launch();
+    using B16 = __nv_bfloat16;
+    kern<<<grid, 256, smem, st>>>(static_cast<const B16*>(q_mask), qcs, qbs, static_cast<const B16*>(k),
+                                  with_v ? static_cast<const B16*>(v) : nullptr, dm.L, dm.Hq, dm.Hkv, dm.flags,
+                                  summary, entropy, with_v ? static_cast<B16*>(o_mask) : nullptr);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)(CONTENT * (D + 1) * (with_v ? 2 : 1) + 8 * D) * sizeof(float);
   auto kern = summary_pool_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
