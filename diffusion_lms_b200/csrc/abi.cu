@@ -685,7 +685,7 @@ rdl_status attn_chunk_major(const void* q, const int32_t* q_pos, const void* k, 
   cm_attn_kernel<<<grid, CM_THREADS, CM_SMEM, st>>>(kmap, vmap, qmap, items, nitems,
                                                    list, dm->Lq, dm->L, dm->Hq, dm->Hkv, dm->K, dm->flags, part);
   const long long n = (long long)dm->B * dm->Lq * dm->Hq;
-  cm_combine_kernel<<<(unsigned)((n + 7) / 8), 256, 0, st>>>(q_pos, idx, z_sel, part, o_loc, lam_loc, nsw, dm->B, dm->L,
+  cm_combine_kernel<<<(unsigned)((n + CM_COMB_WARPS - 1) / CM_COMB_WARPS), CM_COMB_WARPS * 32, 0, st>>>(q_pos, idx, z_sel, part, o_loc, lam_loc, nsw, dm->B, dm->L,
                                                              dm->Lq, dm->Hq, dm->Hkv, dm->K, dm->w, dm->flags,
                                                              static_cast<__nv_bfloat16*>(o), lse);
   return cuda_status(cudaGetLastError());

@@ -455,7 +455,8 @@ __global__ void __launch_bounds__(CM_THREADS, 1)
 // ------------------------------------------------------------------ combine
 // One warp per (b, i, h); lane l owns head dims 4l .. 4l+3.  Window part: nsw key-split
 // planes of (lse, normalised output); chunk parts: the fp16 partials of cm_attn_kernel.
-__global__ void __launch_bounds__(256, 3) cm_combine_kernel(const int32_t* __restrict__ q_pos,
+constexpr int CM_COMB_WARPS = 4;
+__global__ void __launch_bounds__(CM_COMB_WARPS * 32, 3) cm_combine_kernel(const int32_t* __restrict__ q_pos,
                                                          const int32_t* __restrict__ idx,
                                                          const float* __restrict__ z_sel,
                                                          const __half* __restrict__ part,
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(256, 3) cm_combine_kernel(const int32_t* __res
                                                          float* __restrict__ lse) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31;
-  const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const long long item = (long long)blockIdx.x * CM_COMB_WARPS + (threadIdx.x >> 5);
   if (item >= (long long)B * Lq * Hq) return;
   const int h = (int)(item % Hq);
   const int i = (int)((item / Hq) % Lq);
@@ -478,52 +479,75 @@ __global__ void __launch_bounds__(256, 3) cm_combine_kernel(const int32_t* __res
   const size_t li = (size_t)(b * Hq + h) * Lq + i;
   const size_t plane_l = (size_t)B * Hq * Lq, plane_o = (size_t)B * Lq * Hq * D;
   const size_t bg = (size_t)b * Hkv + g;
-  // chunk logits (lanes k, k + 32 hold slot k) and the window planes' lse
-  float zk[2] = {-INFINITY, -INFINITY};
+  // Every load that does not depend on a weight is issued first, so the row costs one memory
+  // round trip: the chunk ids and logits (lanes k, k + 32 hold slot k), the first window
+  // plane, and the chunk outputs of slots 0-31 (a slot without a chunk is read too and gets
+  // weight 0).
   const int32_t* irow = idx + (bg * Lq + i) * K;
   const float* zrow = z_sel + li * K;
+  int ck[2] = {-1, -1};
+  float zr[2] = {-INFINITY, -INFINITY};
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int k = lane + 32 * u;
     if (k < K) {
-      const int c = irow[k];
-      // the same rule as the bucketing kernels (no status recorded a second time)
-      bool on = c >= 0 && c < C;
-      if (on && (flags & RDL_FLAG_CHECKS) && !chunk_eligible(c, p, w)) on = false;
-      if (on) zk[u] = zrow[k];
+      ck[u] = irow[k];
+      zr[u] = zrow[k];
     }
   }
+  const float ls0 = nsw > 0 ? lam_loc[li] : -INFINITY;
+  const float4 vw0 = nsw > 0 ? *reinterpret_cast<const float4*>(o_loc + rh * D + 4 * lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+  const __half* pb = part + ((bg * Lq + i) * K * G + hl) * D + 4 * lane;
+  uint2 raw[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    raw[u] = u < K ? __ldcs(reinterpret_cast<const uint2*>(pb + (size_t)u * G * D)) : make_uint2(0u, 0u);
+  float zk[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    // the same rule as the bucketing kernels (no status recorded a second time)
+    const int c = ck[u];
+    bool on = c >= 0 && c < C;
+    if (on && (flags & RDL_FLAG_CHECKS) && !chunk_eligible(c, p, w)) on = false;
+    if (on) zk[u] = zr[u];
+  }
   float M = warp_max(fmaxf(zk[0], zk[1]));
-  for (int sw = 0; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
+  M = fmaxf(M, ls0);
+  for (int sw = 1; sw < nsw; ++sw) M = fmaxf(M, lam_loc[sw * plane_l + li]);
   if (M == -INFINITY) M = 0.f;
   const float ek0 = zk[0] == -INFINITY ? 0.f : expf(zk[0] - M);
   const float ek1 = zk[1] == -INFINITY ? 0.f : expf(zk[1] - M);
   float Z = warp_sum(ek0 + ek1);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int sw = 0; sw < nsw; ++sw) {
-    const float ls = lam_loc[sw * plane_l + li];
+    const float ls = sw == 0 ? ls0 : lam_loc[sw * plane_l + li];
     if (ls == -INFINITY) continue;
     const float f = expf(ls - M);
     Z += f;
-    const float4 vw = *reinterpret_cast<const float4*>(o_loc + sw * plane_o + rh * D + 4 * lane);
+    const float4 vw = sw == 0 ? vw0 : *reinterpret_cast<const float4*>(o_loc + sw * plane_o + rh * D + 4 * lane);
     acc.x += f * vw.x; acc.y += f * vw.y; acc.z += f * vw.z; acc.w += f * vw.w;
   }
-  const __half* pb = part + ((bg * Lq + i) * K * G + hl) * D + 4 * lane;
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    uint2 raw[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int k = k0 + u;
-      const float f = __shfl_sync(0xffffffffu, (k < 32) ? ek0 : ek1, k & 31);
-      raw[u] = (k < K && f != 0.f) ? __ldcs(reinterpret_cast<const uint2*>(pb + (size_t)k * G * D)) : make_uint2(0u, 0u);
+  for (int u = 0; u < 32; ++u) {
+    const float f = __shfl_sync(0xffffffffu, ek0, u);
+    if (u < K && f != 0.f) {
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].x));
+      const float2 c2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].y));
+      acc.x += f * a.x; acc.y += f * a.y; acc.z += f * c2.x; acc.w += f * c2.y;
     }
+  }
+  for (int k0 = 32; k0 < K; k0 += 8) {        // K > 32: the rest in batches of 8
+    uint2 r8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      r8[u] = k0 + u < K ? __ldcs(reinterpret_cast<const uint2*>(pb + (size_t)(k0 + u) * G * D)) : make_uint2(0u, 0u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int k = k0 + u;
-      const float f = __shfl_sync(0xffffffffu, (k < 32) ? ek0 : ek1, k & 31);
-      if (k < K && f != 0.f) {
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].x));
-        const float2 c2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].y));
+      const float f = __shfl_sync(0xffffffffu, ek1, (k0 + u) & 31);
+      if (k0 + u < K && f != 0.f) {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r8[u].x));
+        const float2 c2 = __half22float2(*reinterpret_cast<const __half2*>(&r8[u].y));
         acc.x += f * a.x; acc.y += f * a.y; acc.z += f * c2.x; acc.w += f * c2.y;
       }
     }
