@@ -621,6 +621,8 @@ def main():
                     help="time only the 28-layer 128K stack (profiling aid)")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the 128K decode block (profiling aid)")
+    ap.add_argument("--prefill-only", choices=["64k", "128k", "16k_k8"], default=None,
+                    help="time only this prefill workload (profiling aid)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -671,6 +673,14 @@ def main():
         dec = decode_bench(args, dev, stream, flush, rank, world, max_ranks, pk, pk_kind)
         if rank == 0:
             print(json.dumps({"decode_128k": dec}), flush=True)
+        return
+    if args.prefill_only:
+        make = {"64k": lambda: W.prefill_64k(seed=rank_seed(4, rank)),
+                "128k": lambda: W.prefill_128k(seed=rank_seed(6, rank)),
+                "16k_k8": lambda: W.prefill_16k_k8(seed=rank_seed(7, rank))}[args.prefill_only]
+        rec = prefill_long_bench(make, args, api, rdl, dev, stream, flush, world, max_ranks, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"prefill_" + args.prefill_only: rec}), flush=True)
         return
 
     # ---------------- 16K prefill route layer (the headline workload)

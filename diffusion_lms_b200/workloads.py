@@ -215,6 +215,8 @@ PREFILL_64K = Dims(B=1, L=65536, Lq=65536, Hq=28, Hkv=4, d=128, D=3584, r=64, K=
                    w=256, lam=0.1, dtype="bf16")
 PREFILL_128K = Dims(B=1, L=131072, Lq=131072, Hq=28, Hkv=4, d=128, D=3584, r=64, K=32,
                     w=256, lam=0.1, dtype="bf16")
+PREFILL_16K_K8 = Dims(B=1, L=16384, Lq=16384, Hq=28, Hkv=4, d=128, D=3584, r=64, K=8,
+                      w=256, lam=0.1, dtype="bf16")
 STACK_LAYERS = 28
 STACK_ROUTE_EVERY = 4          # route layer when layer % 4 == 3
 
@@ -238,6 +240,12 @@ def decode_128k(seed: int = 3) -> Workload:
 def prefill_64k(seed: int = 4) -> Workload:
     """Route layer prefill at 64K with keys from a 32-component mixture (near-tie top-K)."""
     return make_inputs(PREFILL_64K, seed=seed, mixture=32, name="route_prefill_64k_mixture")
+
+
+def prefill_16k_k8(seed: int = 7) -> Workload:
+    """The 16K prefill shapes with K = 8 chunks per query: sparse chunk buckets per row tile,
+    so the selected-chunk attention takes its chunk-major form on a case a few GB in size."""
+    return make_inputs(PREFILL_16K_K8, seed=seed, n_needles=8, name="route_prefill_16k_k8")
 
 
 def prefill_128k(seed: int = 6) -> Workload:
