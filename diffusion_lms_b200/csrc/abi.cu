@@ -319,7 +319,7 @@ rdl_status launch_topk(const float* zeta, const float* z_all, const int32_t* q_p
     return cuda_status(cudaGetLastError());
   }
   const int warps = 4;
-  const size_t smem = (size_t)warps * (C + 256) * sizeof(uint32_t);
+  const size_t smem = (size_t)warps * topk_warp_words(C) * sizeof(uint32_t);
   if (cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return RDL_ERR_CUDA;

@@ -287,11 +287,20 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// One warp per (b, g, i): exact top-K of zeta over the row by a 4-pass 8-bit radix select
-// for the K-th largest key, then one in-order pass that takes every key above it and the
-// first (by chunk index) of the keys equal to it -- ties to the smaller chunk index, and
-// the selection comes out in ascending chunk order.  Then the per-head scores of the
-// selected chunks are gathered.
+// One warp per (b, g, i): exact top-K of zeta over the row, ties to the smaller chunk index,
+// the selection in ascending chunk order; then the per-head scores of the selected chunks are
+// gathered.  Candidate filter first: with packed keys (order key << 32 | ~chunk, distinct per
+// chunk), every lane holds ceil(K/32) keys at or above its ceil(K/32)-th largest, so the
+// smallest of those over the warp bounds the K-th largest key from below and only the keys at
+// or above it (typically a few K) are ranked exactly.  When more than TK_MAXCAND keys pass
+// (heavy near-ties), or the row is short (C < TK_FILTER_MINC), a 4-pass 8-bit radix select finds the K-th largest key and one in-order
+// pass takes every key above it and the first (by chunk index) of the keys equal to it.
+constexpr int TK_MAXCAND = 256;
+constexpr int TK_FILTER_MINC = 512;   // below this many chunks the radix select is faster (measured)
+// shared memory words per warp of topk_radix_kernel: keys [C], then (8-byte aligned) the
+// radix histogram or the packed candidates
+__host__ __device__ inline int topk_warp_words(int C) { return ((C + 1) & ~1) + 2 * TK_MAXCAND; }
+
 __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict__ zeta,
                                                          const float* __restrict__ z_all,
                                                          const int32_t* __restrict__ q_pos, int Lq,
@@ -305,8 +314,8 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
   if (item >= (long long)Lq * Hkv) return;
   const int b = blockIdx.y;
   const int g = (int)(item / Lq), i = (int)(item % Lq);
-  uint32_t* keys = tk_smem + (size_t)warp * (C + 256);
-  uint32_t* hist = keys + C;
+  uint32_t* keys = tk_smem + (size_t)warp * topk_warp_words(C);
+  uint32_t* hist = keys + ((C + 1) & ~1);
   const int p = q_pos ? q_pos[(size_t)b * Lq + i] : i;
   int32_t* irow = idx + ((size_t)(b * Hkv + g) * Lq + i) * K;
   if (is_mask_slot(p)) {
@@ -318,7 +327,18 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
   }
   const float* zr = zeta + ((size_t)(b * Hkv + g) * Lq + i) * C;
   const uint32_t kneg = order_key(-INFINITY);
+  auto packed = [](uint32_t k, int cc) -> unsigned long long {
+    return ((unsigned long long)k << 32) | (0xffffffffu - (uint32_t)cc);
+  };
   int nvalid = 0;
+  unsigned long long m1 = 0ull, m2 = 0ull;     // the lane's two largest packed keys
+  auto track = [&](uint32_t k, int cc) {
+    if (k > kneg) {
+      ++nvalid;
+      const unsigned long long pk = packed(k, cc);
+      if (pk > m1) { m2 = m1; m1 = pk; } else if (pk > m2) { m2 = pk; }
+    }
+  };
   int c = lane;
   for (; c + 7 * 32 < C; c += 8 * 32) {      // 8 independent loads in flight per lane
     float zv[8];
@@ -328,20 +348,72 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
     for (int u = 0; u < 8; ++u) {
       const uint32_t k = order_key(zv[u]);
       keys[c + 32 * u] = k;
-      nvalid += (k > kneg);
+      track(k, c + 32 * u);
     }
   }
   for (; c < C; c += 32) {
     const uint32_t k = order_key(zr[c]);
     keys[c] = k;
-    nvalid += (k > kneg);
+    track(k, c);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
   __syncwarp();
+  int nsel = -1;           // set by the candidate filter when it decides the row
+  if (nvalid > K && K <= 64 && C >= TK_FILTER_MINC) {
+    unsigned long long t0 = K <= 32 ? m1 : m2;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, t0, o);
+      t0 = y < t0 ? y : t0;
+    }
+    // t0 = 0 when a lane holds too few valid keys: then every valid key is a candidate
+    int cnt = 0;
+    for (int cc = lane; cc < C; cc += 32) {
+      const uint32_t k = keys[cc];
+      cnt += (k > kneg && packed(k, cc) >= t0);
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= TK_MAXCAND) {
+      unsigned long long* cand = reinterpret_cast<unsigned long long*>(hist);
+      int pos = incl - cnt;
+      for (int cc = lane; cc < C; cc += 32) {
+        const uint32_t k = keys[cc];
+        if (k > kneg) {
+          const unsigned long long pk = packed(k, cc);
+          if (pk >= t0) cand[pos++] = pk;
+        }
+      }
+      __syncwarp();
+      // exact rank of each candidate (packed keys are distinct); the K best by rank into
+      // selr[0 .. K), then into ascending chunk order
+      int* selr = reinterpret_cast<int*>(keys);     // the keys are no longer read
+      for (int j = lane; j < total; j += 32) {
+        const unsigned long long mine = cand[j];
+        int rank = 0;
+        for (int m = 0; m < total; ++m) rank += cand[m] > mine;
+        if (rank < K) selr[rank] = (int)(0xffffffffu - (uint32_t)(mine & 0xffffffffull));
+      }
+      __syncwarp();
+      for (int j = lane; j < K; j += 32) {
+        const int cj = selr[j];
+        int at = 0;
+        for (int m = 0; m < K; ++m) at += selr[m] < cj;
+        irow[at] = cj;
+      }
+      __syncwarp();
+      nsel = K;
+    }
+  }
   uint32_t thr = kneg;     // take keys > thr, plus `need` keys == thr (smallest indices)
   int need = 0;
-  if (nvalid > K) {
+  if (nsel < 0 && nvalid > K) {
     uint32_t prefix = 0, pmask = 0;
     need = K;
     for (int shift = 24; shift >= 0; shift -= 8) {
@@ -388,7 +460,8 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
     }
     thr = prefix;
   }
-  // in-order selection
+  // in-order selection (unless the candidate filter decided the row)
+  if (nsel < 0) {
   int taken = 0, ties = 0;
   const unsigned lt = (1u << lane) - 1u;
   for (int base = 0; base < C; base += 32) {
@@ -407,7 +480,8 @@ __global__ void __launch_bounds__(128) topk_radix_kernel(const float* __restrict
   }
   for (int k = taken + lane; k < K; k += 32) irow[k] = -1;
   __syncwarp();
-  const int nsel = taken < K ? taken : K;
+  nsel = taken < K ? taken : K;
+  }
   // per-head scores of the selection (without z_all they come later, from the scorer's second
   // pass over the selected chunks; every slot starts at -inf)
   for (int e = lane; e < K * G; e += 32) {

@@ -5,14 +5,16 @@
 //
 // One CTA per (chunk c, KV head g, batch b): the chunk's 63 content keys (and values)
 // are read from HBM once into shared memory and reused by every query head of the group.
-// The pass streams K/V once, so it is HBM-bound.  bf16 inputs take summary_pool_bulk_kernel
-// (one bulk copy per slab, bf16 in shared memory, 32 KB per CTA, so several CTAs per SM keep
-// their copies in flight together); fp32 inputs, or mask-query strides that do not keep a
-// lane's elements aligned, take summary_pool_kernel (fp32 staging).
+// The pass streams K/V once, so it is HBM-bound.  Three forms: bf16 with d = 128 and at most
+// 8 heads per group takes summary_pool_mma_kernel (tensor cores, K/V slabs by TMA); other
+// bf16 shapes take summary_pool_bulk_kernel (one bulk copy per slab, bf16 in shared memory);
+// fp32 inputs, or mask-query strides that do not keep a lane's elements aligned, take
+// summary_pool_kernel (fp32 staging).
 #pragma once
 #include <type_traits>
 #include "common.cuh"
 #include "tc.cuh"
+#include "tmap.cuh"
 
 namespace rdl {
 
@@ -285,6 +287,171 @@ __global__ void __launch_bounds__(256) summary_pool_bulk_kernel(
   }
 }
 
+// bf16, d = 128: the same pooling on tensor cores (mma.sync, fp32 accumulate).  The chunk's K
+// and V slabs arrive by TMA with the 128-byte swizzle (conflict-free ldmatrix); the group's
+// mask queries are the A operand (rows = head slots 0-7, rows 8-15 zero):
+//     logits  L = Q_mask K^T          (16 x 64, exact bf16 products, fp32 sums)
+//     softmax over the 63 content keys per head (quad shuffles), entropy as above
+//     s = a K, o = a V                (a split into bf16 hi + lo terms: s to ~2^-17)
+// CTA = (chunk, KV head, batch), 4 warps: every warp forms the logits and the softmax of all
+// heads (cheap), then the weighted sums for its quarter of the head dimensions.
+constexpr int SPM_THREADS = 128;
+__device__ __forceinline__ uint32_t spm_kv_off(int row, int col) {   // [2 halves][64 rows][128 B]
+  return (uint32_t)((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
+}
+__global__ void __launch_bounds__(SPM_THREADS) summary_pool_mma_kernel(
+    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+    const __nv_bfloat16* __restrict__ q_mask, long long q_chunk_stride, long long q_batch_stride, int with_v,
+    int L, int Hq, int Hkv, int flags, float* __restrict__ summary, float* __restrict__ entropy,
+    __nv_bfloat16* __restrict__ o_mask) {
+  constexpr int D = 128;
+  extern __shared__ unsigned char spm_raw[];
+  unsigned char* sm = spm_raw + ((1024u - (smem_u32(spm_raw) & 1023u)) & 1023u);
+  __shared__ __align__(8) uint64_t bar;
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int C = L / S, G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::mbar_fence_init();
+    const int row0 = (b * Hkv + g) * L + c * S;
+    tc::mbar_arrive_expect_tx(&bar, with_v ? 32768u : 16384u);
+    tc::tma_load_3d(sm, &kmap, 0, row0, 0, &bar);
+    if (with_v) tc::tma_load_3d(sm + 16384, &vmap, 0, row0, 0, &bar);
+  }
+  // A fragments of the mask queries (head slot gq; rows 8-15 of the tile are zero)
+  uint32_t qa[8][2];
+  {
+    const bool on = gq < G;
+    const __nv_bfloat16* qrow = q_mask + (size_t)b * q_batch_stride + (size_t)c * q_chunk_stride + (size_t)(g * G + (on ? gq : 0)) * D;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa[ks][0] = on ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
+      qa[ks][1] = on ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8) : 0u;
+    }
+  }
+  __syncthreads();
+  if (!tc::mbar_wait(&bar, 0)) return;   // bounded; status recorded
+  const uint32_t kst = smem_u32(sm), vst = kst + 16384;
+  const float tau = rsqrtf((float)D);
+  const bool mean = (flags & RDL_FLAG_MEAN_SUMMARY) != 0;
+  // ---- logits (row gq: head slot gq; columns 8 nt + 2 tq + {0, 1}: keys)
+  float sc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+  if (!mean) {
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b0, b1, b2, b3;
+        const int key = 16 * np + 8 * (mi >> 1) + (lane & 7), col = 16 * ks + 8 * (mi & 1);
+        ldsm_x4(kst + spm_kv_off(key, col), b0, b1, b2, b3);
+        mma_bf16(sc[2 * np], a, b0, b1);
+        mma_bf16(sc[2 * np + 1], a, b2, b3);
+      }
+    }
+  }
+  // ---- softmax over the 63 content keys of head slot gq (key 63 is the mask slot)
+  float l[16];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int key = 8 * nt + 2 * tq + e;
+      l[2 * nt + e] = key < CONTENT ? sc[nt][e] * tau : -INFINITY;
+    }
+  float m = l[0];
+#pragma unroll
+  for (int x = 1; x < 16; ++x) m = fmaxf(m, l[x]);
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  float ex[16], z = 0.f;
+#pragma unroll
+  for (int x = 0; x < 16; ++x) {
+    ex[x] = l[x] == -INFINITY ? 0.f : expf(l[x] - m);
+    z += ex[x];
+  }
+  z += __shfl_xor_sync(0xffffffffu, z, 1);
+  z += __shfl_xor_sync(0xffffffffu, z, 2);
+  const float inv = 1.f / z;
+  float sal = 0.f;
+#pragma unroll
+  for (int x = 0; x < 16; ++x) {
+    ex[x] *= inv;                                   // pooling weight a_j
+    if (l[x] != -INFINITY) sal += ex[x] * (l[x] - m);
+  }
+  sal += __shfl_xor_sync(0xffffffffu, sal, 1);
+  sal += __shfl_xor_sync(0xffffffffu, sal, 2);
+  const float H = logf(z) - sal;
+  // ---- A fragments of the weights (split bf16 hi + lo), FA2 layout of the logit tiles
+  uint32_t ph[4][4], pl[4][4];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const float a0 = ex[2 * (2 * kk + half)], a1 = ex[2 * (2 * kk + half) + 1];
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+      ph[kk][2 * half] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+      pl[kk][2 * half] = pack_bf16(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+      ph[kk][2 * half + 1] = 0u;                    // rows 8-15
+      pl[kk][2 * half + 1] = 0u;
+    }
+  }
+  // ---- s = a K and o = a V for head dims [32 warp, 32 warp + 32)
+  float sacc[4][4], oacc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[nt][e] = oacc[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm) {
+      const int key = 16 * kk + 8 * (mi & 1) + (lane & 7), col = 32 * warp + 16 * mm + 8 * (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(kst + spm_kv_off(key, col), b0, b1, b2, b3);
+      mma_bf16(sacc[2 * mm], ph[kk], b0, b1);
+      mma_bf16(sacc[2 * mm], pl[kk], b0, b1);
+      mma_bf16(sacc[2 * mm + 1], ph[kk], b2, b3);
+      mma_bf16(sacc[2 * mm + 1], pl[kk], b2, b3);
+      if (with_v) {
+        ldsm_x4_t(vst + spm_kv_off(key, col), b0, b1, b2, b3);
+        mma_bf16(oacc[2 * mm], ph[kk], b0, b1);
+        mma_bf16(oacc[2 * mm], pl[kk], b0, b1);
+        mma_bf16(oacc[2 * mm + 1], ph[kk], b2, b3);
+        mma_bf16(oacc[2 * mm + 1], pl[kk], b2, b3);
+      }
+    }
+  }
+  if (gq >= G) return;
+  const int h = g * G + gq;
+  float* srow = summary + ((size_t)(b * Hq + h) * C + c) * D;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const int col = 32 * warp + 8 * nt + 2 * tq;
+    if (flags & RDL_FLAG_SPLIT_SUMMARY) {
+      // the same 4D bytes as D bf16 hi terms, then D bf16 lo terms (s = hi + lo)
+      __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(srow);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(sacc[nt][0]), h1 = __float2bfloat16_rn(sacc[nt][1]);
+      *reinterpret_cast<uint32_t*>(hrow + col) = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+      *reinterpret_cast<uint32_t*>(hrow + D + col) =
+          pack_bf16(sacc[nt][0] - __bfloat162float(h0), sacc[nt][1] - __bfloat162float(h1));
+    } else {
+      *reinterpret_cast<float2*>(srow + col) = make_float2(sacc[nt][0], sacc[nt][1]);
+    }
+    if (with_v) {
+      __nv_bfloat16* orow = o_mask + (size_t)b * q_batch_stride + (size_t)c * q_chunk_stride + (size_t)h * D;
+      *reinterpret_cast<uint32_t*>(orow + col) = pack_bf16(oacc[nt][0], oacc[nt][1]);
+    }
+  }
+  if (warp == 0 && tq == 0) entropy[(size_t)(b * Hq + h) * C + c] = H;
+}
+
 template <typename T, int D>
 cudaError_t launch_summary_pool(const void* q_mask, long long qcs, long long qbs, const void* k,
                                 const void* v, const rdl_dims& dm, float* summary, float* entropy,
@@ -294,6 +461,24 @@ cudaError_t launch_summary_pool(const void* q_mask, long long qcs, long long qbs
   // the bulk kernel reads and writes a lane's D/32 mask-query elements as one vector: the
   // strides must keep every mask row aligned to it
   constexpr long long kVec = D / 32;
+  if (std::is_same<T, __nv_bfloat16>::value && D == 128 && dm.Hq / dm.Hkv <= 8 && qcs % 2 == 0 && qbs % 2 == 0) {
+    // tensor-core pooling (the mask-query rows are read as bf16 pairs)
+    CUtensorMap kmap, vmap;
+    const unsigned long long rows = (unsigned long long)dm.B * dm.Hkv * dm.L;
+    if (!make_tmap_kv_halves(&kmap, k, rows) || (with_v && !make_tmap_kv_halves(&vmap, v, rows)))
+      return cudaErrorInvalidValue;
+    if (!with_v) vmap = kmap;
+    const size_t smem = 32768 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(summary_pool_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(C, dm.Hkv, dm.B);
+    count_launch();
+    summary_pool_mma_kernel<<<grid, SPM_THREADS, smem, st>>>(
+        kmap, vmap, static_cast<const __nv_bfloat16*>(q_mask), qcs, qbs, with_v ? 1 : 0, dm.L, dm.Hq, dm.Hkv,
+        dm.flags, summary, entropy, with_v ? static_cast<__nv_bfloat16*>(o_mask) : nullptr);
+    return cudaGetLastError();
+  }
   if (std::is_same<T, __nv_bfloat16>::value && qcs % kVec == 0 && qbs % kVec == 0) {
     const size_t smem = (size_t)CONTENT * D * 2 * (with_v ? 2 : 1);
     auto kern = summary_pool_bulk_kernel<D>;
