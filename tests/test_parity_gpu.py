@@ -327,6 +327,32 @@ def test_prefill_64k_mixture_sampled():
     assert r["n_tie"] > 0          # the mixture keys create near ties
 
 
+def test_prefill_exact_ties_long_rows():
+    """Every eligible chunk of every row ties: zero content queries and hidden states, and the
+    content keys of each chunk all equal (uniform pooling, the same entropy everywhere), so
+    z = -lambda ln 63 for every remote chunk.  512 chunks per row (the prefill top-K's
+    candidate filter path); the selection must be the K lowest eligible chunks (ties to the
+    smaller chunk index) and the outputs must match the oracle on sampled rows."""
+    dm = small(L=32768, Lq=32768, Hq=8, Hkv=2, K=32, w=64)
+    wl = W.make_inputs(dm, seed=37, n_needles=0)
+    wl.q[:] = 0
+    wl.x[:] = 0
+    B, Hkv, L, d = wl.k.shape
+    kc = wl.k.reshape(B, Hkv, L // 64, 64, d)
+    kc[:, :, :, 1:63, :] = kc[:, :, :, 0:1, :]
+    gpu = P.run_gpu(wl)
+    rows = np.unique(np.concatenate([np.arange(0, 200, 7), np.arange(16000, 16200, 9), np.arange(32600, 32768, 5)]))
+    r = P.check_route_layer(wl, gpu, rows)
+    assert r["n_tie"] > 0
+    idx = gpu["idx"][0]
+    for i in (5, 1000, 20000, 32700):
+        if i % 64 == 63:
+            continue
+        wl_lo, wl_hi = max(0, i - 64) // 64, min(L - 1, i + 64) // 64
+        want = [c for c in range(L // 64) if c < wl_lo or c > wl_hi][:32]
+        assert idx[0, i].tolist() == want and idx[1, i].tolist() == want
+
+
 def test_prefill_128k_sampled():
     """Route-layer prefill at 128K: summaries of all 2048 chunks, 512 sampled rows (first
     and last chunks, window edges, rows next to needles), properties on every row."""
